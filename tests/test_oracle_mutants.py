@@ -1,0 +1,75 @@
+"""The oracle pins must catch plausible mistakes.
+
+Each case plants one mistake in a copy of oracle.c (on the CPU, in a temporary
+directory), builds it, and runs the pin suite against that build in a child
+process. Every mutant must fail at least one pin; the unmodified source must pass.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "oracle.c")
+
+# (name, exact text in oracle.c, replacement, occurrence to replace: 0 = first, 1 = second)
+MUTANTS = [
+    ("gate_dropped", "g * oracle_bf16_to_double(xr[c])", "oracle_bf16_to_double(xr[c])", 0),
+    ("residual_sign", "oracle_bf16_to_double(rr[c]) + g *", "oracle_bf16_to_double(rr[c]) - g *", 0),
+    ("norm_on_unrounded_r", "v[c] = oracle_bf16_to_double(rb);", "v[c] = exact;", 0),
+    ("double_rounding_r", "oracle_bf16_rne(exact)", "oracle_bf16_rne((double)(float)exact)", 0),
+    ("eps_outside_sqrt", "1.0 / sqrt(second + eps)", "1.0 / (sqrt(second) + eps)", 0),
+    ("eps_ignored", "1.0 / sqrt(second + eps)", "1.0 / sqrt(second + 1e-5)", 0),
+    ("unbiased_variance", "second /= (double)D;", "second /= (double)(D > 1 ? D - 1 : 1);", 1),
+    ("mean_off_by_one", "mu /= (double)D;", "mu /= (double)(D + 1);", 0),
+    ("rms_uses_abs", "second += v[c] * v[c];", "second += fabs(v[c]);", 0),
+    ("scale_shift_swapped", "(1.0 + oracle_bf16_to_double(sr[c])) + oracle_bf16_to_double(tr[c])",
+     "(1.0 + oracle_bf16_to_double(tr[c])) + oracle_bf16_to_double(sr[c])", 0),
+    ("modulation_without_one", "n * (1.0 + oracle_bf16_to_double(sr[c]))", "n * (oracle_bf16_to_double(sr[c]))", 0),
+    ("weight_added", "n = n * oracle_bf16_to_double(weight[c]);", "n = n + oracle_bf16_to_double(weight[c]);", 0),
+    ("bias_dropped", "n = n + oracle_bf16_to_double(bias[c]);", "n = n;", 0),
+    ("frame_index_mod", "l / tokens_per_frame : 0", "l % tokens_per_frame : 0", 0),
+    ("ties_away", "(frac == 0.5 && fmod(whole, 2.0) == 1.0)", "(frac == 0.5)", 0),
+    ("rounding_truncates", "if (frac > 0.5 || (frac == 0.5 && fmod(whole, 2.0) == 1.0)) whole += 1.0;", "", 0),
+    ("subnormal_quantum", "if (qexp < -133) qexp = -133;", "if (qexp < -126) qexp = -126;", 0),
+]
+
+
+def _apply(text, old, new, occurrence):
+    pos = -1
+    for _ in range(occurrence + 1):
+        pos = text.index(old, pos + 1)
+    return text[:pos] + new + text[pos + len(old):]
+
+
+def _run_pins(lib_path):
+    env = dict(os.environ, ORACLE_LIB=lib_path, OMP_NUM_THREADS="4")
+    cmd = [sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+           os.path.join(ROOT, "tests", "test_oracle_pins.py")]
+    return subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+
+
+def _build(tmp_path, text, name):
+    sys.path.insert(0, ROOT)
+    from oracle.build import build
+
+    src = tmp_path / f"{name}.c"
+    src.write_text(text)
+    return build(str(src), str(tmp_path / f"lib{name}.so"))
+
+
+def test_unmodified_oracle_passes_pins(tmp_path):
+    lib = _build(tmp_path, open(SRC).read(), "clean")
+    res = _run_pins(lib)
+    assert res.returncode == 0, res.stdout[-2000:]
+
+
+@pytest.mark.parametrize("name,old,new,occ", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(tmp_path, name, old, new, occ):
+    text = open(SRC).read()
+    mutated = _apply(text, old, new, occ)
+    assert mutated != text
+    lib = _build(tmp_path, mutated, name)
+    res = _run_pins(lib)
+    assert res.returncode != 0, f"mutant {name} passed every pin:\n{res.stdout[-1500:]}"
