@@ -1,0 +1,488 @@
+"""Benchmark of the fused residual / gate / norm / modulation kernel on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--rows L] [--no-e2e] [--no-cpu-baseline]
+
+One step = one call of the op over the whole workload (every full tensor read or
+written once). Default workload: WAN2.2-shaped LayerNorm, B=1 L=176400 D=5120 bf16,
+gate (1,D), per-row scale/shift, no affine weight (the shape the pages' microbenchmark
+uses: sglang PR #36349, section "Microbenchmark"). Inputs are seeded synthetic
+bf16 values; they are larger than L2 (7.2 GB read per step), so no flush is needed
+between steps.
+
+Metric: achieved HBM GB/s, counting the algorithmic bytes (each full tensor once,
+broadcast operands once), also reported as rows/s and as a fraction of the measured
+HBM copy bandwidth. Multi-GPU: one process per GPU (torchrun); each rank runs its own
+full-size problem (rows are independent, nothing is exchanged), value = all ranks'
+bytes / max-over-ranks time (weak scaling).
+
+--impl reference times the fp64 CPU oracle (the only other implementation that
+exists) on the host cores, on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+import synth.device  # noqa: E402
+
+METRIC = "achieved HBM GB/s (% of B200 peak) and rows/s, fused LN L=176400 D=5120 bf16"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL = "fused_norm_rows"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=1000)
+    p.add_argument("--warmup", type=int, default=50)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=synth.W4.name, choices=sorted(synth.WORKLOADS))
+    p.add_argument("--rows", type=int, default=0, help="override L (profiling a smaller case)")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    return p.parse_args()
+
+
+def workload(args):
+    w = synth.WORKLOADS[args.workload]
+    if args.rows:
+        F = w.F
+        if F and args.rows % F:
+            raise SystemExit(f"--rows must be a multiple of {F} for {w.name}")
+        w = synth.scaled(w, args.rows)
+    return w
+
+
+def config_dict(w, spec, n):
+    lay = {op: w.layout(op) for op in ("gate", "scale", "shift")}
+    return {"workload": w.name, "B": w.B, "L": w.L, "D": w.D, "frames": w.F or None,
+            "norm": "rms" if spec.is_rms else "layer", "has_gate": spec.has_gate,
+            "has_weight": spec.has_weight, "layouts": lay, "eps": w.eps,
+            "parallelism": f"rows per rank, {n} independent problem(s)" if n > 1 else "single GPU",
+            "l2": "inputs larger than L2 (no flush needed)" if w.algorithmic_bytes(spec) > 4 * 126e6
+                  else "L2-resident (small case)"}
+
+
+def kernel_source_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "rmsnorm_row_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            h.update(name.encode())
+            h.update(open(os.path.join(csrc, name), "rb").read())
+    return h.hexdigest()
+
+
+def recorded_traffic(w, spec):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel source; otherwise None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
+    if not m or m.group(1) != kernel_source_digest():
+        return None
+    m = re.search(rf"^{re.escape(w.name)}\s+traffic_bytes_per_launch:\s*([0-9]+)", text, re.M)
+    return int(m.group(1)) if m else None
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_ids):
+        self.lines, self.proc, self.gpu_ids = [], None, gpu_ids
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", ",".join(str(i) for i in self.gpu_ids), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        return self.summary()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for _, line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import rmsnorm_row_b200 as fn
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+
+    w = workload(args)
+    spec = w.specs[0]
+    bytes_step = w.algorithmic_bytes(spec)
+    norm = "rms" if spec.is_rms else "layer"
+
+    # Inputs: generated into pinned host buffers (these are also the e2e host inputs),
+    # then copied to the device once.
+    host = {}
+    for name in ("x", "residual", "gate", "scale", "shift", "weight", "bias"):
+        if name == "gate" and not spec.has_gate or name == "weight" and not spec.has_weight \
+                or name == "bias" and not spec.has_bias:
+            continue
+        n = 1 if name in ("weight", "bias") else w.stored_rows(name)
+        t = torch.empty((n, w.D), dtype=torch.int16, pin_memory=True)
+        w.generate(name, out=t.numpy().view(np.uint16))
+        host[name] = t.view(torch.bfloat16).view(synth.device.operand_view_shape(w, name))
+    d = {k: v.to(dev) for k, v in host.items()}
+    y = torch.empty((w.B, w.L, w.D), dtype=torch.bfloat16, device=dev)
+    r = torch.empty_like(y)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        fn.fused_residual_norm_scale_shift(d["residual"], d["x"], d.get("gate"), d.get("weight"),
+                                           d.get("bias"), d["scale"], d["shift"], norm, w.eps,
+                                           out=y, residual_out=r, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+
+    sampler = ClockSampler([local]) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        t_end = time.time() + 1.0       # keep the GPU busy while nvidia-smi starts
+        while time.time() < t_end:
+            step()
+        torch.cuda.synchronize(dev)
+
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    launches = 0
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev[0].record(stream)
+    for i in range(K):
+        step()
+        launches += 1
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop() if sampler else None
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(K)]
+    total_ms = ev[0].elapsed_time(ev[K])
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_step = total_ms / K
+
+    # e2e: the same op through the public API with host buffers; every step copies
+    # its inputs in from pinned memory and its outputs back, in row chunks on three
+    # streams so copies in, compute and copies out overlap.
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, w, spec, host, d, dev, world, local, fn, torch, dist)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, spec, host, args.cpu_seconds)
+
+    if rank == 0:
+        peak, peak_kind = measured_peak()
+        kernel_ms = statistics.mean(per)
+        achieved = bytes_step / (kernel_ms * 1e-3) / 1e9
+        value = world * bytes_step / (ms_step * 1e-3) / 1e9
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded normal draws, WAN2.2 shapes; no model weights)",
+            "config": config_dict(w, spec, world),
+            "rows_per_s": round(world * w.rows / (ms_step * 1e-3), 1),
+            "pct_of_peak": round(100.0 * value / world / peak, 2),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                         "peak_kind": f"{peak_kind} (HBM copy bandwidth)", "unit": "GB/s",
+                         "frac": round(achieved / peak, 4),
+                         "traffic": recorded_traffic(w, spec), "kernel": KERNEL,
+                         "algorithmic_bytes_per_launch": bytes_step,
+                         "kernel_ms_mean": round(kernel_ms, 5),
+                         "kernel_ms_median": round(statistics.median(per), 5)},
+            "clocks": clocks,
+            "gpu_launches": launches,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_e2e(args, w, spec, host, d, dev, world, local, fn, torch, dist):
+    norm = "rms" if spec.is_rms else "layer"
+    rows = w.rows
+    chunk = 4096
+    hy = torch.empty((w.B, w.L, w.D), dtype=torch.bfloat16, pin_memory=True)
+    hr = torch.empty_like(hy, pin_memory=True)
+    s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    dy = torch.empty((w.B, w.L, w.D), dtype=torch.bfloat16, device=dev)
+    dr = torch.empty_like(dy)
+    per_row = {k: (w.layout(k) == "row") for k in ("gate", "scale", "shift")}
+    flat = lambda t: t.view(-1, w.D)
+    h2d_bytes = sum(v.numel() * 2 for v in host.values())
+    d2h_bytes = (hy.numel() + hr.numel()) * 2
+
+    n_chunks = (rows + chunk - 1) // chunk
+    kernel_done = [None] * n_chunks   # chunk c's kernel of the previous step
+    copied_out = [None] * n_chunks    # chunk c's copy-out of the previous step
+
+    def one():
+        # broadcast / per-frame operands: one small copy per step (after every kernel
+        # of the previous step that reads them)
+        with torch.cuda.stream(s_in):
+            if kernel_done[-1] is not None:
+                s_in.wait_event(kernel_done[-1])
+            for k in ("gate", "scale", "shift", "weight", "bias"):
+                if k in host and not per_row.get(k, False):
+                    d[k].copy_(host[k], non_blocking=True)
+        for c, r0 in enumerate(range(0, rows, chunk)):
+            r1 = min(rows, r0 + chunk)
+            with torch.cuda.stream(s_in):
+                if kernel_done[c] is not None:      # inputs of chunk c no longer read
+                    s_in.wait_event(kernel_done[c])
+                for k in ("x", "residual") + tuple(k for k in ("gate", "scale", "shift") if per_row.get(k)):
+                    flat(d[k])[r0:r1].copy_(flat(host[k])[r0:r1], non_blocking=True)
+                e_in = torch.cuda.Event()
+                e_in.record(s_in)
+            s_cmp.wait_event(e_in)
+            if copied_out[c] is not None:           # outputs of chunk c already on the host
+                s_cmp.wait_event(copied_out[c])
+            sub = lambda t, k: (flat(t)[r0:r1].view(1, r1 - r0, w.D) if per_row.get(k, True) else t)
+            # a chunk of tokens is a (1, n, D) problem when B == 1 and there is no frame axis
+            fn.fused_residual_norm_scale_shift(
+                sub(d["residual"], "residual"), sub(d["x"], "x"),
+                sub(d["gate"], "gate") if "gate" in d else None, d.get("weight"), d.get("bias"),
+                sub(d["scale"], "scale"), sub(d["shift"], "shift"), norm, w.eps,
+                out=flat(dy)[r0:r1].view(1, r1 - r0, w.D),
+                residual_out=flat(dr)[r0:r1].view(1, r1 - r0, w.D), stream=s_cmp)
+            e_c = torch.cuda.Event()
+            e_c.record(s_cmp)
+            kernel_done[c] = e_c
+            s_out.wait_event(e_c)
+            with torch.cuda.stream(s_out):
+                flat(hy)[r0:r1].copy_(flat(dy)[r0:r1], non_blocking=True)
+                flat(hr)[r0:r1].copy_(flat(dr)[r0:r1], non_blocking=True)
+                e_o = torch.cuda.Event()
+                e_o.record(s_out)
+            copied_out[c] = e_o
+
+    if w.B != 1 or w.F:
+        return {"value": None, "unit": "GB/s", "note": "e2e chunking implemented for B=1 without frames"}
+    one()
+    torch.cuda.synchronize(dev)
+    K = max(1, args.e2e_steps)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(s_in)
+    for _ in range(K):
+        one()
+    # the last step's results must be on the host
+    s_in.wait_stream(s_out)
+    t1.record(s_in)
+    torch.cuda.synchronize(dev)
+    ms = t0.elapsed_time(t1) / K
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    return {"value": round(world * w.algorithmic_bytes(spec) / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "ms_per_step": round(ms, 3), "steps": K, "h2d_bytes_per_step": h2d_bytes,
+            "d2h_bytes_per_step": d2h_bytes,
+            "how": "pinned host inputs copied in and outputs copied out every step, 4096-row "
+                   "chunks pipelined over copy-in / compute / copy-out streams"}
+
+
+# ------------------------------------------------------------------ oracle (CPU)
+
+def _oracle_rows(w, spec, host_np, r0, r1):
+    import oracle
+    n = r1 - r0
+    st = (n * w.D, 0, w.D)
+    bst = lambda k: st if w.layout(k) == "row" else (0, 0, 0)
+    sl = lambda k: host_np[k][r0:r1] if w.layout(k) == "row" else host_np[k]
+    return oracle.fused_norm(1, n, w.D, x=host_np["x"][r0:r1], x_st=st,
+                             residual=host_np["residual"][r0:r1], res_st=st,
+                             gate=sl("gate") if spec.has_gate else None,
+                             gate_st=bst("gate") if spec.has_gate else None,
+                             weight=host_np.get("weight"), bias=host_np.get("bias"),
+                             scale=sl("scale"), scale_st=bst("scale"), shift=sl("shift"),
+                             shift_st=bst("shift"), is_rms=spec.is_rms, eps=w.eps)
+
+
+def cpu_baseline(w, spec, host, seconds):
+    """The oracle, as it stands, on the leading rows of the same inputs until about
+    `seconds` of wall time have passed (bounded sample)."""
+    import oracle
+    if w.B != 1 or w.F:
+        return None
+    host_np = {k: v.view(torch_int16()).numpy().view(np.uint16).reshape(-1, w.D) for k, v in host.items()}
+    per_row_bytes = w.algorithmic_bytes(spec) / w.rows
+    done, t0, chunk = 0, time.time(), 1024
+    while time.time() - t0 < seconds and done < w.rows:
+        r1 = min(w.rows, done + chunk)
+        _oracle_rows(w, spec, host_np, done, r1)
+        done = r1
+    el = time.time() - t0
+    return {"value": round(done * per_row_bytes / el / 1e9, 4), "unit": "GB/s",
+            "rows_per_s": round(done / el, 1), "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"first {done} of {w.rows} rows of the same workload ({el:.1f} s)"}
+
+
+def torch_int16():
+    import torch
+    return torch.int16
+
+
+def run_reference(args):
+    """The fp64 oracle on the host cores, K timed steps of a bounded row sample."""
+    import oracle
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    w = workload(args)
+    spec = w.specs[0]
+    if w.B != 1 or w.F:
+        print(json.dumps({"impl": "reference", "unavailable": "reference arm implemented for B=1 workloads"}))
+        return
+    per_row_bytes = w.algorithmic_bytes(spec) / w.rows
+    # size the per-step sample so warm-up + timed steps take about 2 minutes
+    budget_s = 120.0
+    probe_rows = 512
+    names = ["x", "residual", "scale", "shift"] + (["gate"] if spec.has_gate else []) + \
+        (["weight"] if spec.has_weight else []) + (["bias"] if spec.has_bias else [])
+
+    def gen(rows):
+        out = {}
+        for name in names:
+            per_token = name in ("x", "residual") or (name not in ("weight", "bias") and w.layout(name) == "row")
+            out[name] = w.generate(name, np.arange(rows if per_token else 1, dtype=np.int64))
+        return out
+
+    probe = gen(probe_rows)
+    t0 = time.time()
+    _oracle_rows(w, spec, probe, 0, probe_rows)
+    t_row = (time.time() - t0) / probe_rows
+    steps = args.steps + max(args.warmup, 0)
+    rows = int(max(64, min(w.rows, budget_s / max(steps, 1) / max(t_row, 1e-9))))
+    data = gen(rows)
+    for _ in range(args.warmup):
+        _oracle_rows(w, spec, data, 0, rows)
+    t0 = time.time()
+    for _ in range(args.steps):
+        _oracle_rows(w, spec, data, 0, rows)
+    el = time.time() - t0
+    ms = el / max(args.steps, 1) * 1e3
+    value = rows * per_row_bytes / (ms * 1e-3) / 1e9
+    line = {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded normal draws, WAN2.2 shapes)", "impl": "reference",
+            "config": config_dict(w, spec, 1),
+            "rows_per_s": round(rows / (ms * 1e-3), 1),
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": f"first {rows} of {w.rows} rows per step"},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,109 @@
+"""GPU parity: the CUDA kernels (called through the C ABI via the binding) against
+the fp64 oracle on the same seeded inputs.
+
+Workloads are the pages' test matrix and WAN2.2 shapes (sglang PR #33144,
+"Accuracy Tests": every is_rms x has_gate x has_weight, both scale/shift layouts,
+D in {5120, 10240}, L in {16, 90000}, the 4D frame-gate layout; sglang PR #36349,
+"Microbenchmark": LayerNorm at seq 176400, dim 5120). Pass criterion: see
+tests/parity.py (>= 99.99% of y within 1 bf16 ulp, max |err| <= 2e-2, r bit-exact).
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from parity import Tally, check_workload, compare_rows, run_gpu
+from synth.device import upload
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda:0")
+
+
+def _assert(ty: Tally, tr: Tally, label: str):
+    print(f"\n{label}\n  y: {ty}\n  r: {tr}")
+    assert ty.ok(), f"{label}: y fails the tolerance: {ty}"
+    if tr.n:
+        assert tr.exact == tr.n, f"{label}: r not bit-exact: {tr}"
+
+
+def test_gpu_available():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    cap = torch.cuda.get_device_capability(0)
+    assert cap[0] >= 10, f"sm_100a kernels need compute capability 10.x, got {cap}"
+
+
+# ---- small configs: every element -------------------------------------------
+
+def test_rms_fused_B1_L16():
+    w = synth.W1
+    _assert(*check_workload(w, w.specs[0], DEV), w.name)
+
+
+@pytest.mark.parametrize("spec", synth.W2.specs, ids=lambda s: s.name)
+def test_ln_fused_rowgate_B2_L16(spec):
+    w = synth.W2
+    _assert(*check_workload(w, spec, DEV), f"{w.name}/{spec.name}")
+
+
+@pytest.mark.parametrize("D", [5120, 10240])
+@pytest.mark.parametrize("spec", synth._ALL8, ids=lambda s: s.name)
+def test_all_specs_ragged_L(D, spec):
+    # L = 1237 (odd), B = 2: several thousand rows across both batches, outliers included
+    base = synth.W3 if D == 5120 else synth.W3B
+    w = synth.scaled(base, 1237)
+    w = synth.dataclasses.replace(w, B=2, name=f"{w.name}_B2")
+    _assert(*check_workload(w, spec, DEV), f"{w.name}/{spec.name}")
+
+
+@pytest.mark.parametrize("D", [5120, 10240])
+@pytest.mark.parametrize("spec", [synth.Spec(False, True, True, has_bias=True),
+                                  synth.Spec(True, False, False, has_bias=True),
+                                  synth.Spec(False, False, True, norm_only=True),
+                                  synth.Spec(True, False, False, norm_only=True),
+                                  synth.Spec(False, False, True, has_bias=True, norm_only=True)],
+                         ids=lambda s: s.name)
+def test_bias_and_norm_only(D, spec):
+    base = synth.W3 if D == 5120 else synth.W3B
+    w = synth.scaled(base, 777)
+    _assert(*check_workload(w, spec, DEV), f"{w.name}/{spec.name}")
+
+
+@pytest.mark.parametrize("w", [synth.W6, synth.scaled(synth.W5, 420, F=21),
+                               synth.scaled(synth.W5B, 490, F=49)], ids=lambda w: w.name)
+def test_extra_layouts(w):
+    for spec in w.specs:
+        _assert(*check_workload(w, spec, DEV), f"{w.name}/{spec.name}")
+
+
+# ---- full-size configs --------------------------------------------------------
+
+@pytest.mark.parametrize("D", [5120, 10240])
+def test_all_specs_B1_L90000_full(D):
+    w = synth.W3 if D == 5120 else synth.W3B
+    # one upload with every operand; each specialisation reads what it needs
+    dev = upload(w, synth.Spec(False, True, True, has_bias=False), DEV)
+    for spec in w.specs:
+        _assert(*check_workload(w, spec, DEV, dev=dev), f"{w.name}/{spec.name}")
+    del dev
+    torch.cuda.empty_cache()
+
+
+def _full_size(w):
+    spec = w.specs[0]
+    dev = upload(w, spec, DEV)
+    ty, tr = check_workload(w, spec, DEV, dev=dev)
+    del dev
+    torch.cuda.empty_cache()
+    _assert(ty, tr, f"{w.name}/{spec.name}")
+
+
+def test_wan22_ln_B1_L176400_full():
+    _full_size(synth.W4)
+
+
+def test_frame_gate_B1_F21x8400_full():
+    _full_size(synth.W5)
+
+
+def test_frame_gate_B1_F49x3600_full():
+    _full_size(synth.W5B)

@@ -1,0 +1,197 @@
+"""GPU checks that need no oracle run, or that pin the kernel to exact values:
+hand-derived worked cases, closed forms and identities (constant rows, scale = -1,
+gate = 0, gate-free = unit gate), the unfused composition (norm of the returned r
+gives the same y), bitwise determinism and in-place residual update, edge shapes
+(empty, single row, ragged, padded strides) with guard bands, and argument errors
+leaving outputs untouched. All calls go through the C ABI via the binding.
+"""
+import numpy as np
+import pytest
+import torch
+
+import golden_cases
+import oracle
+import rmsnorm_row_b200 as fn
+import synth
+from helpers import ulp_distance
+from parity import Tally
+from synth.device import from_bits, to_bits, upload
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda:0")
+
+
+def bf(a):
+    return torch.as_tensor(np.asarray(a, dtype=np.float32)).to(torch.bfloat16).to(DEV)
+
+
+def rand_bf16(shape, sd=1.0, mu=0.0, seed=0):
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    return (mu + sd * torch.randn(shape, generator=g)).to(torch.bfloat16).to(DEV)
+
+
+def bits(t):
+    return to_bits(t)
+
+
+# ---- hand-derived worked cases (tests/golden/hand_cases.txt), tiled ----------------
+
+@pytest.mark.parametrize("D", [5120, 10240])
+@pytest.mark.parametrize("case", golden_cases.load(), ids=lambda c: c["name"])
+def test_hand_cases_exact(case, D):
+    c = golden_cases.tiled(case, D)
+    L = 3  # several identical rows
+    t = lambda k: from_bits(np.tile(c[k], (1, L, 1)), DEV)
+    res, x = t("residual"), t("x")
+    gate = None if c["gate"] is None else from_bits(c["gate"].reshape(1, 1, D), DEV)
+    scale, shift = t("scale"), t("shift")
+    y, r = fn.fused_residual_norm_scale_shift(res, x, gate, None, None, scale, shift,
+                                              "rms" if c["is_rms"] else "layer", 1e-6)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(r)[0], np.tile(c["want_r"], (L, 1)))
+    assert np.array_equal(bits(y)[0], np.tile(c["want_y"], (L, 1)))
+
+
+# ---- closed forms and identities ------------------------------------------------------
+
+@pytest.mark.parametrize("D", [5120, 10240])
+def test_constant_rows_give_shift_exactly(D):
+    L = 64
+    vals = torch.tensor([0.0, 1.0, -3.5, 0.15625, 96.0, 1e-3, -250.0, 7.0] * 8)[:L]
+    res = vals.view(1, L, 1).expand(1, L, D).to(torch.bfloat16).contiguous().to(DEV)
+    x = rand_bf16((1, L, D), seed=1)
+    gate = torch.zeros((1, 1, D), dtype=torch.bfloat16, device=DEV)
+    scale, shift = rand_bf16((1, L, D), 0.1, seed=2), rand_bf16((1, L, D), 0.1, seed=3)
+    y, r = fn.fused_residual_norm_scale_shift(res, x, gate, None, None, scale, shift, "layer", 1e-6)
+    torch.cuda.synchronize()
+    assert torch.equal(r.view(torch.int16), res.view(torch.int16))          # gate = 0: r = residual
+    assert (ulp_distance(bits(y), bits(shift)) == 0).all()                  # n = 0: y = shift
+
+
+@pytest.mark.parametrize("is_rms", [False, True])
+def test_scale_minus_one_and_gate_identities(is_rms):
+    D, L = 5120, 40
+    norm = "rms" if is_rms else "layer"
+    res, x = rand_bf16((1, L, D), seed=4), rand_bf16((1, L, D), seed=5)
+    gate = rand_bf16((1, 1, D), 0.5, seed=6)
+    shift = rand_bf16((1, L, D), 0.1, seed=7)
+    minus1 = torch.full((1, 1, D), -1.0, dtype=torch.bfloat16, device=DEV)
+    y, _ = fn.fused_residual_norm_scale_shift(res, x, gate, None, None, minus1, shift, norm, 1e-6)
+    assert (ulp_distance(bits(y), bits(shift)) == 0).all()
+    scale = rand_bf16((1, L, D), 0.1, seed=8)
+    ones = torch.ones((1, 1, D), dtype=torch.bfloat16, device=DEV)
+    y1, r1 = fn.fused_residual_norm_scale_shift(res, x, None, None, None, scale, shift, norm, 1e-6)
+    y2, r2 = fn.fused_residual_norm_scale_shift(res, x, ones, None, None, scale, shift, norm, 1e-6)
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    assert torch.equal(r1.view(torch.int16), r2.view(torch.int16))
+
+
+@pytest.mark.parametrize("spec", [synth.Spec(False, True, False), synth.Spec(True, True, True),
+                                  synth.Spec(False, False, True, has_bias=True)], ids=lambda s: s.name)
+def test_unfused_composition(spec):
+    # norm of the returned r, computed by the kernel as a gate-free call with x = 0 and
+    # again as a norm-only call, gives bitwise the same y as the fused call.
+    w = synth.scaled(synth.W3, 300)
+    dev = upload(w, spec, DEV)
+    norm = "rms" if spec.is_rms else "layer"
+    y, r = fn.fused_residual_norm_scale_shift(dev["residual"], dev["x"], dev["gate"] if spec.has_gate else None,
+                                              dev["weight"], dev["bias"], dev["scale"], dev["shift"], norm, 1e-6)
+    zeros = torch.zeros_like(dev["x"])
+    y2, r2 = fn.fused_residual_norm_scale_shift(r, zeros, None, dev["weight"], dev["bias"],
+                                                dev["scale"], dev["shift"], norm, 1e-6)
+    y3 = fn.norm_scale_shift(r, dev["weight"], dev["bias"], dev["scale"], dev["shift"], norm, 1e-6)
+    torch.cuda.synchronize()
+    assert torch.equal(r2.view(torch.int16), r.view(torch.int16))
+    assert torch.equal(y2.view(torch.int16), y.view(torch.int16))
+    assert torch.equal(y3.view(torch.int16), y.view(torch.int16))
+
+
+def test_determinism_and_in_place_residual():
+    w = synth.scaled(synth.W4, 2048)
+    spec = w.specs[0]
+    dev = upload(w, spec, DEV)
+    y1, r1 = fn.fused_residual_norm_scale_shift(dev["residual"], dev["x"], dev["gate"], None, None,
+                                                dev["scale"], dev["shift"], "layer", 1e-6)
+    y2, r2 = fn.fused_residual_norm_scale_shift(dev["residual"], dev["x"], dev["gate"], None, None,
+                                                dev["scale"], dev["shift"], "layer", 1e-6)
+    res_copy = dev["residual"].clone()
+    y3, r3 = fn.fused_residual_norm_scale_shift(res_copy, dev["x"], dev["gate"], None, None,
+                                                dev["scale"], dev["shift"], "layer", 1e-6,
+                                                residual_out=res_copy)
+    torch.cuda.synchronize()
+    assert r3.data_ptr() == res_copy.data_ptr()
+    for a, b in ((y1, y2), (r1, r2), (y1, y3), (r1, res_copy)):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+# ---- edge shapes, strides and guard bands --------------------------------------------
+
+def _padded(B, L, D, pad, fill):
+    """A (B, L, D) view into a bigger buffer with padded rows and canaries around it."""
+    G = 4096  # guard elements on each side
+    buf = torch.full((2 * G + B * L * (D + pad),), fill, dtype=torch.int16, device=DEV)
+    view = buf[G:G + B * L * (D + pad)].view(B, L, D + pad)[:, :, :D].view(torch.bfloat16)
+    return buf, view, G
+
+
+@pytest.mark.parametrize("B,L", [(1, 1), (3, 5), (2, 1), (1, 7)])
+@pytest.mark.parametrize("D", [5120, 10240])
+def test_edge_shapes_padded_outputs_and_guards(B, L, D):
+    res, x = rand_bf16((B, L, D), seed=11), rand_bf16((B, L, D), seed=12)
+    gate = rand_bf16((B, 1, D), 0.5, seed=13)                   # per batch
+    scale, shift = rand_bf16((B, L, D), 0.1, seed=14), rand_bf16((1, 1, D), 0.1, seed=15)
+    weight = rand_bf16((D,), 0.1, 1.0, seed=16)
+    canary = 0x5A5A
+    ybuf, y, G = _padded(B, L, D, 64, canary)
+    rbuf, r, _ = _padded(B, L, D, 128, canary)
+    fn.fused_residual_norm_scale_shift(res, x, gate, weight, None, scale, shift, "layer", 1e-6,
+                                       out=y, residual_out=r)
+    torch.cuda.synchronize()
+    for buf, pad in ((ybuf, 64), (rbuf, 128)):
+        host = buf.cpu().numpy()
+        assert (host[:G] == canary).all() and (host[-G:] == canary).all()
+        body = host[G:len(host) - G].reshape(B, L, D + pad)
+        assert (body[:, :, D:] == canary).all()
+    # values against the oracle
+    xs, rs = bits(x), bits(res)
+    ref = oracle.fused_norm(B, L, D, x=xs, x_st=(L * D, 0, D), residual=rs, res_st=(L * D, 0, D),
+                            gate=bits(gate), gate_st=(D, 0, 0), weight=bits(weight),
+                            scale=bits(scale), scale_st=(L * D, 0, D), shift=bits(shift),
+                            shift_st=(0, 0, 0))
+    ty, tr = Tally(), Tally()
+    ty.add(bits(y.contiguous()), ref["y"])
+    tr.add(bits(r.contiguous()), ref["r"])
+    assert ty.ok(), str(ty)
+    assert tr.exact == tr.n, str(tr)
+
+
+def test_empty_problem_launches_nothing():
+    D = 5120
+    x = torch.empty((0, 16, D), dtype=torch.bfloat16, device=DEV)
+    s = torch.zeros((1, 1, D), dtype=torch.bfloat16, device=DEV)
+    y, r = fn.fused_residual_norm_scale_shift(x.clone(), x, None, None, None, s, s, "layer", 1e-6)
+    assert y.shape == (0, 16, D) and r.shape == (0, 16, D)
+
+
+def test_rejected_call_leaves_outputs_untouched():
+    D, L = 5120, 4
+    res, x = rand_bf16((1, L, D), seed=21), rand_bf16((1, L, D), seed=22)
+    s = torch.zeros((1, 1, D), dtype=torch.bfloat16, device=DEV)
+    y = torch.full((1, L, D), 3.0, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(fn.FusedNormError) as ei:   # y aliases x
+        fn.fused_residual_norm_scale_shift(res, x, None, None, None, s, s, "layer", 1e-6, out=x)
+    assert ei.value.status == fn.FN_ERR_INVALID_ARG
+    raw = torch.zeros(L * D + 8, dtype=torch.bfloat16, device=DEV)
+    mis = raw[1:1 + L * D].view(1, L, D)                          # 2-byte offset
+    with pytest.raises(fn.FusedNormError) as ei:
+        fn.fused_residual_norm_scale_shift(res, mis, None, None, None, s, s, "layer", 1e-6, out=y)
+    assert ei.value.status == fn.FN_ERR_MISALIGNED
+    torch.cuda.synchronize()
+    assert (y.float() == 3.0).all()
+    with pytest.raises(TypeError):
+        fn.fused_residual_norm_scale_shift(res.float(), x, None, None, None, s, s)
+    with pytest.raises(fn.FusedNormError) as ei:
+        fn.fused_residual_norm_scale_shift(res[..., :4096].contiguous(), x[..., :4096].contiguous(),
+                                           None, None, None, s[..., :4096].contiguous(),
+                                           s[..., :4096].contiguous())
+    assert ei.value.status == fn.FN_ERR_UNSUPPORTED
