@@ -19,8 +19,10 @@
  * scale shift" op) has no residual, gate or r: the norm acts on x directly.
  *
  * Data types: every tensor is bf16 (IEEE binary32 truncated to its top 16 bits).
- * Arithmetic is fp32 inside the kernel. eps is a runtime value (the pages' kernel
- * hardcodes 1e-6 and ignores the argument; this library does not).
+ * Arithmetic: fp32 for the element-wise work, fp64 for the row statistics; y is the
+ * correctly rounded bf16 of the formula evaluated with those statistics, and r the
+ * correctly rounded bf16 of the exact residual + gate * x. eps is a runtime value
+ * (the pages' kernel hardcodes 1e-6 and ignores the argument; this library does not).
  *
  * Operand layouts (PR #33144, "Modifications": a broadcast operand is a dense
  * (1, C) row selected for every token; "Accuracy Tests": per-row scale/shift and the
@@ -78,7 +80,7 @@ typedef struct {
   int has_weight; /* 1: n *= weight (affine) */
   int has_bias;   /* 1: n += bias (after the weight) */
   int norm_only;  /* 1: no residual, gate or r; normalise x (requires has_gate == 0) */
-  float eps;      /* added to the variance / mean-square inside the sqrt; finite, >= 0 */
+  double eps;     /* added to the variance / mean-square inside the sqrt; finite, >= 0 */
 } fn_config;
 
 /* One row-addressed bf16 input operand (device pointer). Strides in elements. */

@@ -226,7 +226,7 @@ fn_status fused_norm_create(fused_norm_t* out, const fn_config* cfg) {
   if (!is_flag(c.is_rms) || !is_flag(c.has_gate) || !is_flag(c.has_weight) ||
       !is_flag(c.has_bias) || !is_flag(c.norm_only))
     return FN_ERR_INVALID_ARG;
-  if (!std::isfinite(c.eps) || c.eps < 0.0f) return FN_ERR_INVALID_ARG;
+  if (!std::isfinite(c.eps) || c.eps < 0.0) return FN_ERR_INVALID_ARG;
   if (c.norm_only && c.has_gate) return FN_ERR_INVALID_ARG;
   if (c.D != 5120 && c.D != 10240) return FN_ERR_UNSUPPORTED;
   LaunchFn fn = select_launcher(c.D, c.is_rms, c.norm_only, c.has_gate, c.has_weight, c.has_bias);

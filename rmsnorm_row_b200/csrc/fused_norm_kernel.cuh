@@ -12,18 +12,26 @@
 //     contiguous bytes (fully coalesced 128-bit loads and stores).
 //   * The row stays in registers as packed bf16 between the statistics and the
 //     normalise pass; HBM sees each full tensor exactly once.
-//   * Statistics in fp32: each thread reduces its VPT*8 values locally (two passes
-//     for LayerNorm), warps merge with Chan et al.'s pairwise update through
-//     xor-shuffles (all lanes end bitwise equal), and warps combine through shared
-//     memory in a fixed order after a single barrier. The order never depends on
-//     timing, so results are bitwise reproducible.
+//   * Statistics: every bf16 value is exact in fp64, and so are its square and (for
+//     all practical exponent ranges) the row sums, so each thread accumulates
+//     sum(r) and sum(r^2) in fp64, warps add through xor-shuffles and warps combine
+//     through shared memory in a fixed order after one barrier. LayerNorm takes
+//     var = E[r^2] - mean^2; a row whose mean dwarfs its spread (mean^2 > 2^20 var)
+//     is recomputed with a second, centred pass. The order of every sum is fixed, so
+//     results are bitwise reproducible.
+//   * Output rounding: y is evaluated in fp32 with the fp64 statistics rounded to
+//     fp32, together with a bound on its error (16 units of fp32 roundoff times the
+//     sum of the magnitudes that enter it). When that bound does not reach the
+//     nearest bf16 rounding boundary the fp32 result rounds like the exact value;
+//     otherwise (a few in 10^4 elements) the element is recomputed in fp64 and
+//     rounded once (round-to-odd to fp32, then nearest-even to bf16). y is therefore
+//     the correctly rounded bf16 of the formula evaluated with the fp64 statistics.
+//   * r is the correctly rounded bf16 of the exact residual + gate * x: gate * x is
+//     exact in fp32 (two 8-bit significands); when the fp32 sum lands exactly on a
+//     bf16 midpoint, TwoSum recovers the sum's rounding error and its sign decides.
 //   * Per-row (streamed-once) operands use evict-first loads and stores; broadcast
 //     and per-frame operands use the read-only cached path (they are re-read by
 //     every row and stay in L1/L2).
-//   * r is the correctly rounded bf16 of the exact residual + gate * x: gate * x is
-//     exact in fp32 (two 8-bit significands), TwoSum recovers the error of the fp32
-//     sum, and a sum that lands exactly on a bf16 midpoint is resolved by the sign of
-//     that error instead of ties-to-even.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -49,7 +57,7 @@ struct RowParams {
   int64_t shift_sb, shift_sf, shift_sl;
   int64_t y_sb, y_sl, r_sb, r_sl;
   int64_t L, tpf, rows;
-  float eps;
+  double eps;
   uint32_t stream_mask;  // bit set: operand is per-row (read once) -> streaming load
 };
 
@@ -64,6 +72,42 @@ __device__ __forceinline__ uint4 load_vec(const uint16_t* base, int j, bool stre
 
 __device__ __forceinline__ float lo_f(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float hi_f(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+__device__ __forceinline__ uint32_t word(const uint4& v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+// element q (0..7) of a 16-byte vector of bf16, as fp32
+__device__ __forceinline__ float elem(const uint4& v, int q) {
+  return (q & 1) ? hi_f(word(v, q >> 1)) : lo_f(word(v, q >> 1));
+}
+
+// ---- bf16 arithmetic on packed pairs (sm_90+ bf16x2, sm_100 mixed precision) ----
+
+// d = a * b + c per bf16 lane, the exact result rounded once to nearest-even bf16.
+__device__ __forceinline__ uint32_t fma_bf16x2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+// bf16 half H (0: low, 1: high) of p, plus an fp32 value, rounded once to fp32.
+template <int H>
+__device__ __forceinline__ float add_bf16_f32(uint32_t p, float c) {
+  float d;
+  if (H == 0)
+    asm("{.reg .b16 l, h; mov.b32 {l, h}, %1; add.rn.f32.bf16 %0, l, %2;}" : "=f"(d) : "r"(p), "f"(c));
+  else
+    asm("{.reg .b16 l, h; mov.b32 {l, h}, %1; add.rn.f32.bf16 %0, h, %2;}" : "=f"(d) : "r"(p), "f"(c));
+  return d;
+}
+// bf16 half H of p, exactly, as fp64.
+template <int H>
+__device__ __forceinline__ double bf16_f64(uint32_t p) {
+  double d;
+  if (H == 0)
+    asm("{.reg .b16 l, h; mov.b32 {l, h}, %1; cvt.f64.bf16 %0, l;}" : "=d"(d) : "r"(p));
+  else
+    asm("{.reg .b16 l, h; mov.b32 {l, h}, %1; cvt.f64.bf16 %0, h;}" : "=d"(d) : "r"(p));
+  return d;
+}
 
 __device__ __forceinline__ uint32_t pack_rn(float lo, float hi) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
@@ -72,42 +116,149 @@ __device__ __forceinline__ uint32_t pack_rn(float lo, float hi) {
   return u;
 }
 
-// bf16 bits of (a + p) rounded once to nearest even, where a + p is the exact real
-// sum of two fp32 values (Knuth's TwoSum gives s + e == a + p exactly).
-__device__ __forceinline__ uint32_t round_sum_bf16(float a, float p) {
-  const float s = __fadd_rn(a, p);
-  const float bv = __fsub_rn(s, a);
-  const float av = __fsub_rn(s, bv);
-  const float e = __fadd_rn(__fsub_rn(a, av), __fsub_rn(p, bv));
-  const uint32_t u = __float_as_uint(s);
-  const uint32_t rn = __bfloat16_as_ushort(__float2bfloat16_rn(s));
-  // s sits on a bf16 midpoint but the exact sum does not (e != 0, not NaN):
-  // round towards the exact value.
-  const bool tie = ((u & 0xFFFFu) == 0x8000u) && (fabsf(e) > 0.0f);
-  const uint32_t toward = ((e > 0.0f) == (s > 0.0f)) ? ((u + 0x8000u) >> 16) : (u >> 16);
-  return tie ? toward : rn;
+__device__ __forceinline__ uint32_t bf16_rn(float f) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
 
-// r pair = residual pair + gate pair * x pair
-template <bool HAS_GATE>
-__device__ __forceinline__ uint32_t residual_pair(uint32_t res, uint32_t x, uint32_t g) {
-  float plo = lo_f(x), phi = hi_f(x);
-  if (HAS_GATE) {
-    plo = __fmul_rn(lo_f(g), plo);  // exact: 8-bit x 8-bit significands
-    phi = __fmul_rn(hi_f(g), phi);
-  }
-  return round_sum_bf16(lo_f(res), plo) | (round_sum_bf16(hi_f(res), phi) << 16);
+// bf16 bits of an fp64 value rounded once to nearest even: round to odd into fp32
+// (24 significant bits, at least two more than bf16 needs), then to nearest even.
+__device__ __forceinline__ uint32_t bf16_from_double(double v) {
+  float f = __double2float_rz(v);
+  if ((double)f != v) f = __uint_as_float(__float_as_uint(f) | 1u);
+  return bf16_rn(f);
 }
+
+// One 16-byte vector of r = residual + gate * x (gate = 1 when absent): one bf16x2
+// fused multiply-add per pair gives the exact sum rounded once to bf16.
+template <bool HAS_GATE>
+__device__ __forceinline__ uint4 residual_vec(const uint4& res, const uint4& x, const uint4& g) {
+  constexpr uint32_t kOnes = 0x3F803F80u;  // (1.0, 1.0) in bf16
+  return make_uint4(fma_bf16x2(HAS_GATE ? g.x : kOnes, x.x, res.x),
+                    fma_bf16x2(HAS_GATE ? g.y : kOnes, x.y, res.y),
+                    fma_bf16x2(HAS_GATE ? g.z : kOnes, x.z, res.z),
+                    fma_bf16x2(HAS_GATE ? g.w : kOnes, x.w, res.w));
+}
+
+struct RowStats {
+  double mu, rho;       // fp64 statistics (mu = 0 for RMSNorm)
+  float neg_mu32, rho32;  // -mu and rho rounded to fp32, for the fast path
+  float kappa;          // |mu32| * rho32: how much of n the mean's rounding can move
+};
+
+// y of one element, exactly rounded (see the header comment).
+template <bool HAS_WEIGHT, bool HAS_BIAS>
+__device__ __forceinline__ uint32_t y_exact(float v, float w, float b, float s, float t,
+                                         double mu, double rho) {
+  double n = __dmul_rn(__dsub_rn((double)v, mu), rho);
+  if (HAS_WEIGHT) n = __dmul_rn(n, (double)w);
+  if (HAS_BIAS) n = __dadd_rn(n, (double)b);
+  const double y = __dadd_rn(__dmul_rn(n, __dadd_rn(1.0, (double)s)), (double)t);
+  return bf16_from_double(y);
+}
+
+// fp32 evaluation of y for element q of a vector and whether it is far enough from
+// the bf16 rounding boundary to be rounded as is.
+//
+// Error bound, to first order in u = 2^-24 (mu, rho exact to far better than u):
+// rounding mu and rho to fp32, the subtraction, the product with rho, the weight
+// product, the bias sum, 1 + scale and the final fma each add at most u times one of
+// |1+s| |w| kappa, |1+s| |n w|, |1+s| |n w + b|, |n w + b|, |y|, all of which are at
+// most P = |1+s| (|w| kappa + |n w| + |b|) + |shift|. The sum is at most 8 u P; the
+// test uses 16 u P to cover second-order terms and the rounding of P itself.
+template <int H, bool HAS_WEIGHT, bool HAS_BIAS>
+__device__ __forceinline__ float y_fast(uint32_t vw, uint32_t sw, uint32_t tw, uint32_t ww,
+                                        uint32_t bw, const RowStats& st, bool& near) {
+  constexpr float k16u = 9.5367431640625e-7f;  // 2^-20
+  const float n = add_bf16_f32<H>(vw, st.neg_mu32) * st.rho32;
+  const float w = H ? hi_f(ww) : lo_f(ww);
+  const float nw = HAS_WEIGHT ? n * w : n;
+  const float b = H ? hi_f(bw) : lo_f(bw);
+  const float nb = HAS_BIAS ? nw + b : nw;
+  const float a = add_bf16_f32<H>(sw, 1.0f);
+  const float t = H ? hi_f(tw) : lo_f(tw);
+  const float y = fmaf(nb, a, t);
+  float inner = HAS_WEIGHT ? fmaf(fabsf(w), st.kappa, fabsf(nw)) : st.kappa + fabsf(nw);
+  if (HAS_BIAS) inner += fabsf(b);
+  const float bound = fmaf(fabsf(a), inner, fabsf(t)) * k16u;
+  // the bf16 rounding boundary next to y: same sign and exponent, low half 0x8000
+  const float mid = __uint_as_float((__float_as_uint(y) & 0xFFFF0000u) | 0x8000u);
+  near = near || !(fabsf(y - mid) > bound);  // NaN/Inf also take the fp64 path
+  return y;
+}
+
+// Repair of one vector whose fast path came near a rounding boundary (a rolled loop,
+// so the rarely taken code stays small).
+template <bool HAS_WEIGHT, bool HAS_BIAS>
+__device__ __forceinline__ uint4 y_repair(const uint4& v, const uint4& sv, const uint4& tv,
+                                          const uint4& wv, const uint4& bv, const RowStats& st) {
+  uint32_t h[8];
+#pragma unroll 1
+  for (int q = 0; q < 8; ++q) {
+    const uint32_t vw = word(v, q >> 1), sw = word(sv, q >> 1), tw = word(tv, q >> 1);
+    const uint32_t ww = word(wv, q >> 1), bw = word(bv, q >> 1);
+    bool near = false;
+    const float y = (q & 1) ? y_fast<1, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, ww, bw, st, near)
+                            : y_fast<0, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, ww, bw, st, near);
+    h[q] = near ? y_exact<HAS_WEIGHT, HAS_BIAS>(elem(v, q), elem(wv, q), elem(bv, q), elem(sv, q),
+                                                elem(tv, q), st.mu, st.rho)
+                : bf16_rn(y);
+  }
+  return make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16),
+                    h[6] | (h[7] << 16));
+}
+
+// One 16-byte vector of y.
+template <bool HAS_WEIGHT, bool HAS_BIAS>
+__device__ __forceinline__ uint4 output_vec(const uint4& v, const uint4& sv, const uint4& tv,
+                                            const uint4& wv, const uint4& bv, const RowStats& st) {
+  bool near = false;
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t vw = word(v, i), sw = word(sv, i), tw = word(tv, i);
+    const uint32_t ww = word(wv, i), bw = word(bv, i);
+    const float y0 = y_fast<0, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, ww, bw, st, near);
+    const float y1 = y_fast<1, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, ww, bw, st, near);
+    o[i] = pack_rn(y0, y1);
+  }
+  uint4 out = make_uint4(o[0], o[1], o[2], o[3]);
+  if (near) out = y_repair<HAS_WEIGHT, HAS_BIAS>(v, sv, tv, wv, bv, st);  // rare
+  return out;
+}
+
+// Launch shape per D: vectors per thread (threads = D / (8 VPT)) and the CTAs per SM
+// the register budget is sized for (65536 / (threads * kMinBlocks) registers each).
+template <int D> struct RowShape;
+#ifndef FN_VPT_5120
+#define FN_VPT_5120 5
+#endif
+#ifndef FN_MINB_5120
+#define FN_MINB_5120 5
+#endif
+#ifndef FN_VPT_10240
+#define FN_VPT_10240 4
+#endif
+#ifndef FN_MINB_10240
+#define FN_MINB_10240 2
+#endif
+// 1: scale/shift loads are issued with x and residual, before the r stores;
+// 0: after them, where the statistics' reduction and barrier hide their latency
+// (fewer live registers; measured faster on B200 for the WAN2.2 shape).
+#ifndef FN_EARLY_MODULATION_LOADS
+#define FN_EARLY_MODULATION_LOADS 0
+#endif
+template <> struct RowShape<5120> { static constexpr int VPT = FN_VPT_5120, kMinBlocks = FN_MINB_5120; };
+template <> struct RowShape<10240> { static constexpr int VPT = FN_VPT_10240, kMinBlocks = FN_MINB_10240; };
 
 template <int D, int VPT, bool IS_RMS, bool NORM_ONLY, bool HAS_GATE, bool HAS_WEIGHT, bool HAS_BIAS>
-__global__ void __launch_bounds__(D / (8 * VPT)) fused_norm_rows(const RowParams p) {
+__global__ void __launch_bounds__(D / (8 * VPT), RowShape<D>::kMinBlocks) fused_norm_rows(const RowParams p) {
   constexpr int T = D / (8 * VPT);
   constexpr int W = T / 32;
-  constexpr int PER_THREAD = VPT * 8;
   static_assert(T % 32 == 0 && T * 8 * VPT == D, "row must split evenly into warps");
   static_assert(!(NORM_ONLY && HAS_GATE), "norm-only has no gate");
 
-  __shared__ float2 part[2][W];
+  __shared__ double2 part[2][W];
+  __shared__ double centred[W];
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   int parity = 0;
@@ -121,9 +272,10 @@ __global__ void __launch_bounds__(D / (8 * VPT)) fused_norm_rows(const RowParams
     const uint16_t* sr = p.scale + (b * p.scale_sb + f * p.scale_sf + l * p.scale_sl);
     const uint16_t* tr = p.shift + (b * p.shift_sb + f * p.shift_sf + l * p.shift_sl);
 
-    // ---- loads: every streamed operand is requested before the first store, so
-    // the row's whole input is in flight at once (stores could alias loads as far
-    // as the compiler knows, so loads written after them would wait for them).
+    // ---- loads: x, residual and gate are requested together. scale and shift are
+    // requested with them or right after the r stores (FN_EARLY_MODULATION_LOADS);
+    // a load written after a store waits for the store's issue, since the compiler
+    // cannot rule out aliasing.
     uint4 xv[VPT], rv[VPT], gv[VPT], sv[VPT], tv[VPT];
 #pragma unroll
     for (int k = 0; k < VPT; ++k) xv[k] = load_vec(xr, tid + k * T, p.stream_mask & kX);
@@ -137,97 +289,99 @@ __global__ void __launch_bounds__(D / (8 * VPT)) fused_norm_rows(const RowParams
 #pragma unroll
       for (int k = 0; k < VPT; ++k) gv[k] = load_vec(gr, tid + k * T, p.stream_mask & kGate);
     }
+    if (FN_EARLY_MODULATION_LOADS) {
 #pragma unroll
-    for (int k = 0; k < VPT; ++k) {
-      sv[k] = load_vec(sr, tid + k * T, p.stream_mask & kScale);
-      tv[k] = load_vec(tr, tid + k * T, p.stream_mask & kShift);
+      for (int k = 0; k < VPT; ++k) {
+        sv[k] = load_vec(sr, tid + k * T, p.stream_mask & kScale);
+        tv[k] = load_vec(tr, tid + k * T, p.stream_mask & kShift);
+      }
     }
 
     // ---- step 1: r = residual + gate * x, rounded to bf16, stored -------------
-    uint32_t v[VPT][4];  // the row (r, or x when norm-only), packed bf16 pairs
+    uint4 v[VPT];  // the row (r, or x when norm-only), packed bf16 pairs
     if (NORM_ONLY) {
 #pragma unroll
-      for (int k = 0; k < VPT; ++k) {
-        v[k][0] = xv[k].x; v[k][1] = xv[k].y; v[k][2] = xv[k].z; v[k][3] = xv[k].w;
-      }
+      for (int k = 0; k < VPT; ++k) v[k] = xv[k];
     } else {
       uint4* ro = reinterpret_cast<uint4*>(p.r + (b * p.r_sb + l * p.r_sl));
 #pragma unroll
       for (int k = 0; k < VPT; ++k) {
-        const uint4 g = HAS_GATE ? gv[k] : make_uint4(0, 0, 0, 0);
-        v[k][0] = residual_pair<HAS_GATE>(rv[k].x, xv[k].x, g.x);
-        v[k][1] = residual_pair<HAS_GATE>(rv[k].y, xv[k].y, g.y);
-        v[k][2] = residual_pair<HAS_GATE>(rv[k].z, xv[k].z, g.z);
-        v[k][3] = residual_pair<HAS_GATE>(rv[k].w, xv[k].w, g.w);
-        __stcs(ro + tid + k * T, make_uint4(v[k][0], v[k][1], v[k][2], v[k][3]));
+        v[k] = residual_vec<HAS_GATE>(rv[k], xv[k], HAS_GATE ? gv[k] : rv[k]);
+        __stcs(ro + tid + k * T, v[k]);
       }
     }
 
-    // ---- step 2: row statistics --------------------------------------------
-    float mean = 0.0f, second;
-    if (IS_RMS) {
-      float ss = 0.0f;
+    if (!FN_EARLY_MODULATION_LOADS) {
 #pragma unroll
-      for (int k = 0; k < VPT; ++k)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float a = lo_f(v[k][q]), c = hi_f(v[k][q]);
-          ss = fmaf(a, a, ss);
-          ss = fmaf(c, c, ss);
-        }
-#pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
-      if (lane == 0) part[parity][warp] = make_float2(ss, 0.0f);
-      __syncthreads();
-      float tot = part[parity][0].x;
-#pragma unroll
-      for (int w = 1; w < W; ++w) tot += part[parity][w].x;
-      second = tot / (float)D;
-    } else {
-      float sum = 0.0f;
-#pragma unroll
-      for (int k = 0; k < VPT; ++k)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) sum += lo_f(v[k][q]) + hi_f(v[k][q]);
-      float m = sum / (float)PER_THREAD;
-      float m2 = 0.0f;
-#pragma unroll
-      for (int k = 0; k < VPT; ++k)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float a = lo_f(v[k][q]) - m, c = hi_f(v[k][q]) - m;
-          m2 = fmaf(a, a, m2);
-          m2 = fmaf(c, c, m2);
-        }
-      // Chan's pairwise merge of equal-count partials; symmetric in the two lanes.
-      float half_cnt = 0.5f * (float)PER_THREAD;
-#pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) {
-        const float om = __shfl_xor_sync(0xFFFFFFFFu, m, o);
-        const float om2 = __shfl_xor_sync(0xFFFFFFFFu, m2, o);
-        const float d = om - m;
-        m = (m + om) * 0.5f;
-        m2 = (m2 + om2) + (d * d) * half_cnt;
-        half_cnt *= 2.0f;
+      for (int k = 0; k < VPT; ++k) {
+        sv[k] = load_vec(sr, tid + k * T, p.stream_mask & kScale);
+        tv[k] = load_vec(tr, tid + k * T, p.stream_mask & kShift);
       }
-      if (lane == 0) part[parity][warp] = make_float2(m, m2);
-      __syncthreads();
-      // Warps in a fixed order; every thread computes the same result.
-      constexpr float kWarpCnt = 32.0f * PER_THREAD;
-      float2 acc = part[parity][0];
-#pragma unroll
-      for (int w = 1; w < W; ++w) {
-        const float2 o = part[parity][w];
-        const float na = kWarpCnt * (float)w;
-        const float frac = kWarpCnt / (na + kWarpCnt);
-        const float d = o.x - acc.x;
-        acc.x = acc.x + d * frac;
-        acc.y = (acc.y + o.y) + (d * d) * (na * frac);
-      }
-      mean = acc.x;
-      second = acc.y / (float)D;
     }
-    const float rho = 1.0f / sqrtf(second + p.eps);
+
+    // ---- step 2: row statistics in fp64 ------------------------------------
+    // Four independent accumulation chains per thread (one per word of a vector),
+    // combined in a fixed order: short dependency chains, reproducible sums.
+    double a1[4] = {0.0, 0.0, 0.0, 0.0}, a2[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+    for (int k = 0; k < VPT; ++k)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const double a = bf16_f64<0>(word(v[k], i)), c = bf16_f64<1>(word(v[k], i));
+        if (!IS_RMS) a1[i] += a + c;                 // a + c exact: two bf16 values
+        a2[i] += fma(a, a, c * c);                   // c * c exact (16-bit significand)
+      }
+    double s1 = (a1[0] + a1[1]) + (a1[2] + a1[3]);
+    double s2 = (a2[0] + a2[1]) + (a2[2] + a2[3]);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      if (!IS_RMS) s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, o);
+      s2 += __shfl_xor_sync(0xFFFFFFFFu, s2, o);
+    }
+    if (lane == 0) part[parity][warp] = make_double2(s1, s2);
+    __syncthreads();
+    double t1 = part[parity][0].x, t2 = part[parity][0].y;
+#pragma unroll
+    for (int w = 1; w < W; ++w) {
+      t1 += part[parity][w].x;
+      t2 += part[parity][w].y;
+    }
+    constexpr double kInvD = 1.0 / (double)D;
+    RowStats st;
+    if (IS_RMS) {
+      st.mu = 0.0;
+      st.rho = rsqrt(t2 * kInvD + p.eps);
+    } else {
+      const double mu = t1 * kInvD;
+      double var = fmax(t2 * kInvD - mu * mu, 0.0);
+      if (mu * mu > 1048576.0 * var && var > 0.0) {
+        // The mean dwarfs the spread: take the variance around the mean instead
+        // (uniform branch: every thread of the CTA has the same statistics).
+        double c2 = 0.0;
+#pragma unroll
+        for (int k = 0; k < VPT; ++k)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const double a = bf16_f64<0>(word(v[k], i)) - mu, c = bf16_f64<1>(word(v[k], i)) - mu;
+            c2 = fma(a, a, c2);
+            c2 = fma(c, c, c2);
+          }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) c2 += __shfl_xor_sync(0xFFFFFFFFu, c2, o);
+        if (lane == 0) centred[warp] = c2;
+        __syncthreads();
+        double tc = centred[0];
+#pragma unroll
+        for (int w = 1; w < W; ++w) tc += centred[w];
+        var = tc * kInvD;
+        __syncthreads();  // centred[] is reused by the next such row
+      }
+      st.mu = mu;
+      st.rho = rsqrt(var + p.eps);
+    }
+    st.neg_mu32 = -(float)st.mu;
+    st.rho32 = (float)st.rho;
+    st.kappa = fabsf(st.neg_mu32) * st.rho32;
 
     // ---- step 3: normalise, affine, modulate, store y ------------------------
     uint4* yo = reinterpret_cast<uint4*>(p.y + (b * p.y_sb + l * p.y_sl));
@@ -237,30 +391,7 @@ __global__ void __launch_bounds__(D / (8 * VPT)) fused_norm_rows(const RowParams
       uint4 wv = make_uint4(0, 0, 0, 0), bv = make_uint4(0, 0, 0, 0);
       if (HAS_WEIGHT) wv = __ldg(reinterpret_cast<const uint4*>(p.weight) + j);
       if (HAS_BIAS) bv = __ldg(reinterpret_cast<const uint4*>(p.bias) + j);
-      const uint32_t sw[4] = {sv[k].x, sv[k].y, sv[k].z, sv[k].w};
-      const uint32_t tw[4] = {tv[k].x, tv[k].y, tv[k].z, tv[k].w};
-      const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
-      const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
-      uint32_t out[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float n0 = (lo_f(v[k][q]) - mean) * rho;
-        float n1 = (hi_f(v[k][q]) - mean) * rho;
-        if (HAS_WEIGHT && HAS_BIAS) {
-          n0 = fmaf(n0, lo_f(ww[q]), lo_f(bw[q]));
-          n1 = fmaf(n1, hi_f(ww[q]), hi_f(bw[q]));
-        } else if (HAS_WEIGHT) {
-          n0 *= lo_f(ww[q]);
-          n1 *= hi_f(ww[q]);
-        } else if (HAS_BIAS) {
-          n0 += lo_f(bw[q]);
-          n1 += hi_f(bw[q]);
-        }
-        const float y0 = fmaf(n0, 1.0f + lo_f(sw[q]), lo_f(tw[q]));
-        const float y1 = fmaf(n1, 1.0f + hi_f(sw[q]), hi_f(tw[q]));
-        out[q] = pack_rn(y0, y1);
-      }
-      __stcs(yo + j, make_uint4(out[0], out[1], out[2], out[3]));
+      __stcs(yo + j, output_vec<HAS_WEIGHT, HAS_BIAS>(v[k], sv[k], tv[k], wv, bv, st));
     }
   }
 }
@@ -272,11 +403,6 @@ cudaError_t launch_rows(const RowParams& p, int64_t grid, cudaStream_t stream) {
       <<<(unsigned)grid, T, 0, stream>>>(p);
   return cudaGetLastError();
 }
-
-// Threads per row and vectors per thread, per D.
-template <int D> struct RowShape;
-template <> struct RowShape<5120> { static constexpr int VPT = 4; };
-template <> struct RowShape<10240> { static constexpr int VPT = 4; };
 
 // Launcher for a specialisation, selected at create time. Defined in one
 // translation unit per (D, norm type) so the instances compile in parallel.

@@ -130,10 +130,13 @@ def test_valid_args_pass_and_plan():
     a = valid_args()
     assert fn.fused_norm_validate(h, a) == OK
     st, grid, block, smem = fn.fused_norm_plan(h, a)
-    assert (st, grid, block, smem) == (OK, 16, 160, 0)
+    # one CTA per row; a whole number of warps, each thread owning whole 16-byte vectors
+    assert (st, grid, smem) == (OK, 16, 0)
+    assert block % 32 == 0 and 5120 % (8 * block) == 0
     h2 = make(D=10240)
     st, grid, block, smem = fn.fused_norm_plan(h2, valid_args(D=10240, B=1, L=90000))
-    assert (st, grid, block) == (OK, 90000, 320)
+    assert (st, grid) == (OK, 90000)
+    assert block % 32 == 0 and 10240 % (8 * block) == 0
 
 
 def _mut(**kw):
