@@ -12,8 +12,7 @@ import pytest
 import torch
 
 import synth
-from parity import Tally, check_workload, compare_rows, run_gpu
-from synth.device import upload
+from parity import Tally, check_workload, host_inputs, run_gpu, upload_host
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda:0")
@@ -80,19 +79,21 @@ def test_extra_layouts(w):
 @pytest.mark.parametrize("D", [5120, 10240])
 def test_all_specs_B1_L90000_full(D):
     w = synth.W3 if D == 5120 else synth.W3B
-    # one upload with every operand; each specialisation reads what it needs
-    dev = upload(w, synth.Spec(False, True, True, has_bias=False), DEV)
+    # inputs generated and uploaded once; each specialisation reads what it needs
+    host = host_inputs(w, ("x", "residual", "gate", "scale", "shift", "weight"))
+    dev = upload_host(w, host, DEV)
     for spec in w.specs:
-        _assert(*check_workload(w, spec, DEV, dev=dev), f"{w.name}/{spec.name}")
+        _assert(*check_workload(w, spec, DEV, dev=dev, host=host), f"{w.name}/{spec.name}")
     del dev
     torch.cuda.empty_cache()
 
 
 def _full_size(w):
     spec = w.specs[0]
-    dev = upload(w, spec, DEV)
-    ty, tr = check_workload(w, spec, DEV, dev=dev)
-    del dev
+    host = host_inputs(w, ("x", "residual", "gate", "scale", "shift", "weight"))
+    dev = upload_host(w, host, DEV)
+    ty, tr = check_workload(w, spec, DEV, dev=dev, host=host)
+    del dev, host
     torch.cuda.empty_cache()
     _assert(ty, tr, f"{w.name}/{spec.name}")
 
