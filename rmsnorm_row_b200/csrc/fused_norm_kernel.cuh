@@ -20,7 +20,7 @@
 //     is recomputed with a second, centred pass. The order of every sum is fixed, so
 //     results are bitwise reproducible.
 //   * Output rounding: y is evaluated in fp32 with the fp64 statistics rounded to
-//     fp32, together with a bound on its error (16 units of fp32 roundoff times the
+//     fp32, together with a bound on its error (8 units of fp32 roundoff times the
 //     sum of the magnitudes that enter it). When that bound does not reach the
 //     nearest bf16 rounding boundary the fp32 result rounds like the exact value;
 //     otherwise (a few in 10^4 elements) the element is recomputed in fp64 and
@@ -156,19 +156,23 @@ __device__ __forceinline__ uint32_t y_exact(float v, float w, float b, float s, 
   return bf16_from_double(y);
 }
 
-// fp32 evaluation of y for element q of a vector and whether it is far enough from
-// the bf16 rounding boundary to be rounded as is.
+// fp32 evaluation of y for one element, and whether it is far enough from every bf16
+// rounding boundary to be rounded as is (otherwise `near` is set).
 //
-// Error bound, to first order in u = 2^-24 (mu, rho exact to far better than u):
-// rounding mu and rho to fp32, the subtraction, the product with rho, the weight
-// product, the bias sum, 1 + scale and the final fma each add at most u times one of
-// |1+s| |w| kappa, |1+s| |n w|, |1+s| |n w + b|, |n w + b|, |y|, all of which are at
-// most P = |1+s| (|w| kappa + |n w| + |b|) + |shift|. The sum is at most 8 u P; the
-// test uses 16 u P to cover second-order terms and the rounding of P itself.
+// Error of the fp32 evaluation, to first order in u = 2^-24 (mu and rho are exact to
+// far better than u). With exact n* = (v - mu) rho, the eight roundings (-mu, rho,
+// the subtraction, the product with rho, the weight product, the bias sum, 1 + scale,
+// the final fma) give
+//   |y - y*| <= u (|1+s| |w| kappa + 7 |1+s| |n* w| + 3 |1+s| |b| + |shift|) <= 7 u P,
+//   P = |1+s| (|w| kappa + |n w| + |b|) + |shift|,  kappa = |mu| rho.
+// The test uses B = 8 u P, which also covers second-order terms and P's own rounding.
+// Rounding boundaries next to y: the midpoint D away in its bf16 interval, and, when y
+// lies in the lowest interval of a binade, one at least ulp/4 below (ulp = bf16 spacing
+// at y; |y| 2^-10 <= ulp/4). So y rounds correctly if B < min(D, |y| 2^-10).
 template <int H, bool HAS_WEIGHT, bool HAS_BIAS>
 __device__ __forceinline__ float y_fast(uint32_t vw, uint32_t sw, uint32_t tw, uint32_t ww,
                                         uint32_t bw, const RowStats& st, bool& near) {
-  constexpr float k16u = 9.5367431640625e-7f;  // 2^-20
+  constexpr float k8u = 4.76837158203125e-7f;  // 2^-21
   const float n = add_bf16_f32<H>(vw, st.neg_mu32) * st.rho32;
   const float w = H ? hi_f(ww) : lo_f(ww);
   const float nw = HAS_WEIGHT ? n * w : n;
@@ -179,10 +183,11 @@ __device__ __forceinline__ float y_fast(uint32_t vw, uint32_t sw, uint32_t tw, u
   const float y = fmaf(nb, a, t);
   float inner = HAS_WEIGHT ? fmaf(fabsf(w), st.kappa, fabsf(nw)) : st.kappa + fabsf(nw);
   if (HAS_BIAS) inner += fabsf(b);
-  const float bound = fmaf(fabsf(a), inner, fabsf(t)) * k16u;
+  const float bound = fmaf(fabsf(a), inner, fabsf(t)) * k8u;
   // the bf16 rounding boundary next to y: same sign and exponent, low half 0x8000
   const float mid = __uint_as_float((__float_as_uint(y) & 0xFFFF0000u) | 0x8000u);
-  near = near || !(fabsf(y - mid) > bound);  // NaN/Inf also take the fp64 path
+  const float room = fminf(fabsf(y - mid), fabsf(y) * 9.765625e-4f);  // 2^-10
+  near |= !(room > bound);  // NaN/Inf also take the fp64 path
   return y;
 }
 
