@@ -139,6 +139,19 @@ __device__ __forceinline__ uint4 residual_vec(const uint4& res, const uint4& x, 
                     fma_bf16x2(HAS_GATE ? g.w : kOnes, x.w, res.w));
 }
 
+// a / D rounded once to nearest, for D = 5 * 2^k. Markstein's correction: with
+// y = RN(1/5) and q0 = RN(a y) (within one ulp of a/5), the residual r = a - 5 q0 is
+// exact under fma, and RN(q0 + r y) is the correctly rounded a/5; the power-of-two
+// scaling is then exact. Same result as an IEEE division, without its slow path.
+template <int D>
+__device__ __forceinline__ double div_by_row_length(double a) {
+  static_assert(D == 5120 || D == 10240, "D must be 5 * 2^k");
+  constexpr double kScale = D == 5120 ? 1.0 / 1024.0 : 1.0 / 2048.0;
+  const double q0 = __dmul_rn(a, 0.2);
+  const double r = fma(-5.0, q0, a);
+  return fma(r, 0.2, q0) * kScale;
+}
+
 struct RowStats {
   double mu, rho;       // fp64 statistics (mu = 0 for RMSNorm)
   float neg_mu32, rho32;  // -mu and rho rounded to fp32, for the fast path
@@ -255,8 +268,20 @@ template <int D> struct RowShape;
 template <> struct RowShape<5120> { static constexpr int VPT = FN_VPT_5120, kMinBlocks = FN_MINB_5120; };
 template <> struct RowShape<10240> { static constexpr int VPT = FN_VPT_10240, kMinBlocks = FN_MINB_10240; };
 
+// CTAs per SM the register budget targets for one specialisation. D = 5120 LayerNorm
+// with an affine weight or bias needs more registers than 5 CTAs allow without spills;
+// measured on B200 (L = 90000 and the frame-gate shape), 4 CTAs is faster there, while
+// every other D = 5120 specialisation is faster at 5.
+template <int D, bool IS_RMS, bool HAS_WEIGHT, bool HAS_BIAS>
+struct MinBlocks {
+  static constexpr int value =
+      (D == 5120 && !IS_RMS && (HAS_WEIGHT || HAS_BIAS) && RowShape<D>::kMinBlocks > 4)
+          ? 4 : RowShape<D>::kMinBlocks;
+};
+
 template <int D, int VPT, bool IS_RMS, bool NORM_ONLY, bool HAS_GATE, bool HAS_WEIGHT, bool HAS_BIAS>
-__global__ void __launch_bounds__(D / (8 * VPT), RowShape<D>::kMinBlocks) fused_norm_rows(const RowParams p) {
+__global__ void __launch_bounds__(D / (8 * VPT), (MinBlocks<D, IS_RMS, HAS_WEIGHT, HAS_BIAS>::value))
+fused_norm_rows(const RowParams p) {
   constexpr int T = D / (8 * VPT);
   constexpr int W = T / 32;
   static_assert(T % 32 == 0 && T * 8 * VPT == D, "row must split evenly into warps");
@@ -351,14 +376,16 @@ __global__ void __launch_bounds__(D / (8 * VPT), RowShape<D>::kMinBlocks) fused_
       t1 += part[parity][w].x;
       t2 += part[parity][w].y;
     }
-    constexpr double kInvD = 1.0 / (double)D;
+    // Correctly rounded divisions by D (not products with 1/D): the mean is then the
+    // rounded quotient of the exact sum, as defined, and a row whose mean dwarfs its
+    // spread does not turn a last-bit difference of the mean into a different output.
     RowStats st;
     if (IS_RMS) {
       st.mu = 0.0;
-      st.rho = rsqrt(t2 * kInvD + p.eps);
+      st.rho = rsqrt(div_by_row_length<D>(t2) + p.eps);
     } else {
-      const double mu = t1 * kInvD;
-      double var = fmax(t2 * kInvD - mu * mu, 0.0);
+      const double mu = div_by_row_length<D>(t1);
+      double var = fmax(div_by_row_length<D>(t2) - mu * mu, 0.0);
       if (mu * mu > 1048576.0 * var && var > 0.0) {
         // The mean dwarfs the spread: take the variance around the mean instead
         // (uniform branch: every thread of the CTA has the same statistics).
@@ -378,7 +405,7 @@ __global__ void __launch_bounds__(D / (8 * VPT), RowShape<D>::kMinBlocks) fused_
         double tc = centred[0];
 #pragma unroll
         for (int w = 1; w < W; ++w) tc += centred[w];
-        var = tc * kInvD;
+        var = div_by_row_length<D>(tc);
         __syncthreads();  // centred[] is reused by the next such row
       }
       st.mu = mu;

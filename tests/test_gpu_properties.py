@@ -195,3 +195,50 @@ def test_rejected_call_leaves_outputs_untouched():
                                            None, None, None, s[..., :4096].contiguous(),
                                            s[..., :4096].contiguous())
     assert ei.value.status == fn.FN_ERR_UNSUPPORTED
+
+
+# ---- rounding-boundary and statistics stress ------------------------------------------
+
+def _near_cancelling_problem(D, L, seed, offset=0.0, spread=1.0, is_rms=False):
+    """Rows where shift nearly cancels n * (1 + scale) (so y is tiny and sits close to
+    rounding boundaries), with a mean offset and spread per row; built from the oracle's
+    own n on CPU."""
+    from helpers import f32_to_bf16_bits_rne
+    rng = np.random.default_rng(seed)
+    def bfbits(a):
+        return f32_to_bf16_bits_rne(np.asarray(a, dtype=np.float32))
+    res = bfbits(offset + spread * rng.normal(size=(1, L, D)))
+    x = bfbits(rng.normal(size=(1, L, D)))
+    gate = bfbits(0.5 * rng.normal(size=(1, 1, D)))
+    scale = bfbits(0.3 * rng.normal(size=(1, L, D)))
+    zeros = np.zeros((1, L, D), np.uint16)
+    st = (L * D, 0, D)
+    base = oracle.fused_norm(1, L, D, x=x, x_st=st, residual=res, res_st=st, gate=gate,
+                             gate_st=(0, 0, 0), scale=zeros, scale_st=st, shift=zeros, shift_st=st,
+                             is_rms=is_rms, want_n=True)
+    from helpers import bf16_bits_to_f64
+    s = bf16_bits_to_f64(scale)
+    target = -base["n"] * (1.0 + s) * (1.0 + 1e-3 * rng.normal(size=(1, L, D)))
+    shift = bfbits(target)
+    return res, x, gate, scale, shift
+
+
+@pytest.mark.parametrize("is_rms", [False, True])
+@pytest.mark.parametrize("offset,spread", [(0.0, 1.0), (1000.0, 0.01), (0.0, 1e-3), (-3.0, 40.0)])
+def test_near_cancellation_and_offsets_bit_exact(is_rms, offset, spread):
+    D, L = 5120, 96
+    res, x, gate, scale, shift = _near_cancelling_problem(D, L, 31, offset, spread, is_rms)
+    dev = lambda a: from_bits(a, DEV)
+    y, r = fn.fused_residual_norm_scale_shift(dev(res), dev(x), dev(gate), None, None, dev(scale),
+                                              dev(shift), "rms" if is_rms else "layer", 1e-6)
+    torch.cuda.synchronize()
+    st = (L * D, 0, D)
+    ref = oracle.fused_norm(1, L, D, x=x, x_st=st, residual=res, res_st=st, gate=gate,
+                            gate_st=(0, 0, 0), scale=scale, scale_st=st, shift=shift, shift_st=st,
+                            is_rms=is_rms)
+    ty, tr = Tally(), Tally()
+    ty.add(bits(y), ref["y"])
+    tr.add(bits(r), ref["r"])
+    print(f"\nnear-cancellation offset={offset} spread={spread} rms={is_rms}\n  y: {ty}\n  r: {tr}")
+    assert tr.exact == tr.n
+    assert ty.hist.get(0, 0) == ty.n, f"y not bit-exact: {ty}"
