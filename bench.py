@@ -55,11 +55,26 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default=synth.W4.name, choices=sorted(synth.WORKLOADS))
     p.add_argument("--rows", type=int, default=0, help="override L (profiling a smaller case)")
+    p.add_argument("--spec", default="", help="specialisation of the workload (e.g. rms_gate_w); "
+                   "default: the workload's first")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--graph", action="store_true",
+                   help="replay the timed launches from one CUDA graph (removes host launch "
+                        "overhead; for the launch-bound small shapes)")
     return p.parse_args()
+
+
+def pick_spec(w, args):
+    if not args.spec:
+        return w.specs[0]
+    for sp in w.specs:
+        if sp.name == args.spec:
+            return sp
+    raise SystemExit(f"{w.name} has no specialisation {args.spec!r}; "
+                     f"choose from {[sp.name for sp in w.specs]}")
 
 
 def workload(args):
@@ -74,7 +89,7 @@ def workload(args):
 
 def config_dict(w, spec, n):
     lay = {op: w.layout(op) for op in ("gate", "scale", "shift")}
-    return {"workload": w.name, "B": w.B, "L": w.L, "D": w.D, "frames": w.F or None,
+    return {"workload": w.name, "spec": spec.name, "B": w.B, "L": w.L, "D": w.D, "frames": w.F or None,
             "norm": "rms" if spec.is_rms else "layer", "has_gate": spec.has_gate,
             "has_weight": spec.has_weight, "layouts": lay, "eps": w.eps,
             "parallelism": f"rows per rank, {n} independent problem(s)" if n > 1 else "single GPU",
@@ -190,7 +205,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
 
     w = workload(args)
-    spec = w.specs[0]
+    spec = pick_spec(w, args)
     bytes_step = w.algorithmic_bytes(spec)
     norm = "rms" if spec.is_rms else "layer"
 
@@ -210,10 +225,23 @@ def run_ours(args):
     r = torch.empty_like(y)
     stream = torch.cuda.current_stream(dev)
 
+    # The C arguments are marshalled once; each step is one fused_norm_launch call
+    # (the tensor-level API marshals the same arguments on every call, which costs
+    # ~15 us of host time and dominates the launch-bound small shapes).
+    args_c = fn.build_args(d["x"], d["residual"], d.get("gate"), d.get("weight"), d.get("bias"),
+                           d["scale"], d["shift"], y, r)
+    handle = fn.api._handle(w.D, spec.is_rms, spec.has_gate, spec.has_weight, spec.has_bias,
+                            spec.norm_only, w.eps)
+
     def step():
-        fn.fused_residual_norm_scale_shift(d["residual"], d["x"], d.get("gate"), d.get("weight"),
-                                           d.get("bias"), d["scale"], d["shift"], norm, w.eps,
-                                           out=y, residual_out=r, stream=stream)
+        st = fn.fused_norm_launch(handle, args_c, int(stream.cuda_stream))
+        if st != fn.FN_OK:
+            raise fn.FusedNormError(st, "fused_norm_launch", fn.fused_norm_status_string(st))
+
+    # one call through the tensor-level API first: same result as the prebuilt launch
+    fn.fused_residual_norm_scale_shift(d["residual"], d["x"], d.get("gate"), d.get("weight"),
+                                       d.get("bias"), d["scale"], d["shift"], norm, w.eps,
+                                       out=y, residual_out=r, stream=stream)
 
     def barrier():
         if world > 1:
@@ -234,17 +262,39 @@ def run_ours(args):
     K = args.steps
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
     launches = 0
+    graph = None
+    if args.graph:
+        # capture the K timed launches (no per-step events inside a graph)
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            stream_saved, stream = stream, cap
+            with torch.cuda.graph(graph, stream=cap):
+                for _ in range(K):
+                    step()
+            stream = stream_saved
+        torch.cuda.synchronize(dev)
+        graph.replay()
+        torch.cuda.synchronize(dev)
     barrier()
     torch.cuda.synchronize(dev)
     ev[0].record(stream)
-    for i in range(K):
-        step()
-        launches += 1
-        ev[i + 1].record(stream)
+    if graph is not None:
+        with torch.cuda.stream(stream):
+            graph.replay()
+        launches = K
+        ev[K].record(stream)
+    else:
+        for i in range(K):
+            step()
+            launches += 1
+            ev[i + 1].record(stream)
     torch.cuda.synchronize(dev)
     barrier()
     clocks = sampler.stop() if sampler else None
-    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(K)]
+    per = ([ev[0].elapsed_time(ev[K]) / K] * K if graph is not None
+           else [ev[i].elapsed_time(ev[i + 1]) for i in range(K)])
     total_ms = ev[0].elapsed_time(ev[K])
     t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
     if world > 1:
@@ -273,7 +323,7 @@ def run_ours(args):
             "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded normal draws, WAN2.2 shapes; no model weights)",
-            "config": config_dict(w, spec, world),
+            "config": dict(config_dict(w, spec, world), launch="cuda_graph" if graph is not None else "stream"),
             "rows_per_s": round(world * w.rows / (ms_step * 1e-3), 1),
             "pct_of_peak": round(100.0 * value / world / peak, 2),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
@@ -430,7 +480,7 @@ def run_reference(args):
     if rank != 0:
         return
     w = workload(args)
-    spec = w.specs[0]
+    spec = pick_spec(w, args)
     if w.B != 1 or w.F:
         print(json.dumps({"impl": "reference", "unavailable": "reference arm implemented for B=1 workloads"}))
         return
