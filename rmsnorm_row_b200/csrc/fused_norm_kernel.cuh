@@ -204,43 +204,46 @@ __device__ __forceinline__ float y_fast(uint32_t vw, uint32_t sw, uint32_t tw, u
   return y;
 }
 
-// Repair of one vector whose fast path came near a rounding boundary (a rolled loop,
-// so the rarely taken code stays small).
-template <bool HAS_WEIGHT, bool HAS_BIAS>
-__device__ __forceinline__ uint4 y_repair(const uint4& v, const uint4& sv, const uint4& tv,
-                                          const uint4& wv, const uint4& bv, const RowStats& st) {
-  uint32_t h[8];
-#pragma unroll 1
-  for (int q = 0; q < 8; ++q) {
-    const uint32_t vw = word(v, q >> 1), sw = word(sv, q >> 1), tw = word(tv, q >> 1);
-    const uint32_t ww = word(wv, q >> 1), bw = word(bv, q >> 1);
-    bool near = false;
-    const float y = (q & 1) ? y_fast<1, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, ww, bw, st, near)
-                            : y_fast<0, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, ww, bw, st, near);
-    h[q] = near ? y_exact<HAS_WEIGHT, HAS_BIAS>(elem(v, q), elem(wv, q), elem(bv, q), elem(sv, q),
-                                                elem(tv, q), st.mu, st.rho)
-                : bf16_rn(y);
-  }
-  return make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16),
-                    h[6] | (h[7] << 16));
+// Element q's value from a 16-byte vector, for a runtime q (rare paths only).
+__device__ __forceinline__ float elem_dyn(const uint4& v, int q) {
+  const uint32_t w = q < 2 ? v.x : q < 4 ? v.y : q < 6 ? v.z : v.w;
+  return (q & 1) ? hi_f(w) : lo_f(w);
 }
 
-// One 16-byte vector of y.
+// One 16-byte vector of y: the fp32 fast path for all eight elements, then (rarely) the
+// fp64 path for the elements whose fast value came near a rounding boundary.
 template <bool HAS_WEIGHT, bool HAS_BIAS>
 __device__ __forceinline__ uint4 output_vec(const uint4& v, const uint4& sv, const uint4& tv,
                                             const uint4& wv, const uint4& bv, const RowStats& st) {
-  bool near = false;
   uint32_t o[4];
+  uint32_t near_mask = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const uint32_t vw = word(v, i), sw = word(sv, i), tw = word(tv, i);
     const uint32_t ww = word(wv, i), bw = word(bv, i);
-    const float y0 = y_fast<0, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, ww, bw, st, near);
-    const float y1 = y_fast<1, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, ww, bw, st, near);
+    bool n0 = false, n1 = false;
+    const float y0 = y_fast<0, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, ww, bw, st, n0);
+    const float y1 = y_fast<1, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, ww, bw, st, n1);
     o[i] = pack_rn(y0, y1);
+    near_mask |= (n0 ? 1u : 0u) << (2 * i);
+    near_mask |= (n1 ? 2u : 0u) << (2 * i);
   }
   uint4 out = make_uint4(o[0], o[1], o[2], o[3]);
-  if (near) out = y_repair<HAS_WEIGHT, HAS_BIAS>(v, sv, tv, wv, bv, st);  // rare
+#pragma unroll 1
+  while (near_mask) {  // rare
+    const int q = __ffs(near_mask) - 1;
+    near_mask &= near_mask - 1;
+    const uint32_t bits = y_exact<HAS_WEIGHT, HAS_BIAS>(
+        elem_dyn(v, q), HAS_WEIGHT ? elem_dyn(wv, q) : 1.0f, HAS_BIAS ? elem_dyn(bv, q) : 0.0f,
+        elem_dyn(sv, q), elem_dyn(tv, q), st.mu, st.rho);
+    const uint32_t put = (q & 1) ? (bits << 16) : bits;
+    const uint32_t keep = (q & 1) ? 0x0000FFFFu : 0xFFFF0000u;
+    const int i = q >> 1;
+    out.x = i == 0 ? ((out.x & keep) | put) : out.x;
+    out.y = i == 1 ? ((out.y & keep) | put) : out.y;
+    out.z = i == 2 ? ((out.z & keep) | put) : out.z;
+    out.w = i == 3 ? ((out.w & keep) | put) : out.w;
+  }
   return out;
 }
 
