@@ -251,7 +251,8 @@ def run_ours(args):
         step()
     torch.cuda.synchronize(dev)
 
-    sampler = ClockSampler([local]) if rank == 0 else None
+    # rank 0 samples every GPU of this node that the job uses
+    sampler = ClockSampler(list(range(world))) if rank == 0 else None
     if sampler:
         sampler.start()
         t_end = time.time() + 1.0       # keep the GPU busy while nvidia-smi starts
