@@ -231,7 +231,7 @@ def run_ours(args):
     args_c = fn.build_args(d["x"], d["residual"], d.get("gate"), d.get("weight"), d.get("bias"),
                            d["scale"], d["shift"], y, r)
     handle = fn.api._handle(w.D, spec.is_rms, spec.has_gate, spec.has_weight, spec.has_bias,
-                            spec.norm_only, w.eps)
+                            spec.norm_only, w.eps, False)
 
     def step():
         st = fn.fused_norm_launch(handle, args_c, int(stream.cuda_stream))

@@ -18,7 +18,10 @@
  * value the caller gets back). Norm-only mode (norm_only = 1, the pages' "norm
  * scale shift" op) has no residual, gate or r: the norm acts on x directly.
  *
- * Data types: every tensor is bf16 (IEEE binary32 truncated to its top 16 bits).
+ * Data types: every tensor is bf16 (IEEE binary32 truncated to its top 16 bits), except
+ * that the affine weight and bias may be fp32 (affine_fp32; the pages' kernel takes fp32
+ * affine parameters but casts them to bf16 -- PR 33144, "Known gaps" -- here they are used
+ * at full precision).
  * Arithmetic: fp32 for the element-wise work, fp64 for the row statistics; y is the
  * correctly rounded bf16 of the formula evaluated with those statistics, and r the
  * correctly rounded bf16 of the exact residual + gate * x. eps is a runtime value
@@ -80,6 +83,8 @@ typedef struct {
   int has_weight; /* 1: n *= weight (affine) */
   int has_bias;   /* 1: n += bias (after the weight) */
   int norm_only;  /* 1: no residual, gate or r; normalise x (requires has_gate == 0) */
+  int affine_fp32; /* 1: weight and bias are fp32 (D floats each), used at full precision;
+                      0: bf16. Needs has_weight or has_bias. */
   double eps;     /* added to the variance / mean-square inside the sqrt; finite, >= 0 */
 } fn_config;
 
@@ -97,8 +102,8 @@ typedef struct {
   fn_operand residual;       /* required unless norm_only; NULL when norm_only */
   fn_operand gate;           /* NULL iff has_gate == 0 */
   fn_operand scale, shift;   /* required */
-  const void* weight;        /* (D) contiguous bf16; NULL iff has_weight == 0 */
-  const void* bias;          /* (D) contiguous bf16; NULL iff has_bias == 0 */
+  const void* weight;        /* (D) contiguous bf16 (fp32 if affine_fp32); NULL iff has_weight == 0 */
+  const void* bias;          /* (D) contiguous bf16 (fp32 if affine_fp32); NULL iff has_bias == 0 */
   void* y;                   /* output (B, L, D) bf16: row (b, l) at y + b*y_stride_b + l*y_stride_l */
   int64_t y_stride_b, y_stride_l;
   void* r;                   /* output, same addressing; NULL when norm_only */
@@ -108,7 +113,8 @@ typedef struct {
 /*
  * Create a handle for one specialisation.
  * Errors: FN_ERR_INVALID_ARG (null pointers, flags not 0/1, eps negative or not
- * finite, norm_only with has_gate), FN_ERR_UNSUPPORTED (D not 5120 or 10240).
+ * finite, norm_only with has_gate, affine_fp32 without weight or bias),
+ * FN_ERR_UNSUPPORTED (D not 5120 or 10240).
  * *out is set only on FN_OK. Host only; makes no CUDA call.
  */
 fn_status fused_norm_create(fused_norm_t* out, const fn_config* cfg);

@@ -44,7 +44,7 @@ def _load():
     lib.oracle_bf16_to_double.restype = dbl
     lib.oracle_bf16_rne.argtypes = [dbl]
     lib.oracle_bf16_rne.restype = ctypes.c_uint16
-    lib.oracle_fused_norm.argtypes = [i64, i64, i64, i64, ctypes.c_int, ctypes.c_int, dbl] + [vp] * 18
+    lib.oracle_fused_norm.argtypes = [i64, i64, i64, i64, ctypes.c_int, ctypes.c_int, dbl] + [vp] * 20
     lib.oracle_fused_norm.restype = ctypes.c_int
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ctypes.c_int
@@ -85,6 +85,14 @@ def _bf16_array(a):
     return a
 
 
+def _f32_array(a):
+    if a is None:
+        return None
+    a = np.ascontiguousarray(a)
+    assert a.dtype == np.float32, a.dtype
+    return a
+
+
 def fused_norm(B: int, L: int, D: int, *, x, x_st, scale, scale_st, shift, shift_st,
                residual=None, res_st=None, gate=None, gate_st=None, weight=None, bias=None,
                is_rms: bool = False, norm_only: bool = False, eps: float = 1e-6,
@@ -92,14 +100,18 @@ def fused_norm(B: int, L: int, D: int, *, x, x_st, scale, scale_st, shift, shift
     """Run the oracle over all B*L rows.
 
     Operand arrays are flat-indexable uint16 buffers addressed with strides
-    {stride_b, stride_f, stride_l} in elements (0 = broadcast). Returns a dict with
+    {stride_b, stride_f, stride_l} in elements (0 = broadcast). weight and bias are
+    (D,) uint16 bf16 bit patterns or (D,) float32 arrays. Returns a dict with
     ``y`` (B, L, D) uint16, ``r`` (B, L, D) uint16 or None, and optionally ``n``
     (B, L, D) float64 (the normalised value before the affine step) and ``stats``
     (B*L, 3) float64 (mean or 0, variance or mean-square, 1/sqrt(. + eps)).
     """
     lib = _load()
     x, residual, gate = _bf16_array(x), _bf16_array(residual), _bf16_array(gate)
-    weight, bias = _bf16_array(weight), _bf16_array(bias)
+    w16 = _bf16_array(weight) if weight is not None and np.asarray(weight).dtype == np.uint16 else None
+    b16 = _bf16_array(bias) if bias is not None and np.asarray(bias).dtype == np.uint16 else None
+    w32 = _f32_array(weight) if weight is not None and w16 is None else None
+    b32 = _f32_array(bias) if bias is not None and b16 is None else None
     scale, shift = _bf16_array(scale), _bf16_array(shift)
     y = np.empty((B, L, D), dtype=np.uint16)
     r = None if norm_only else np.empty((B, L, D), dtype=np.uint16)
@@ -112,7 +124,7 @@ def fused_norm(B: int, L: int, D: int, *, x, x_st, scale, scale_st, shift, shift
     rc = lib.oracle_fused_norm(
         B, L, D, tokens_per_frame, int(bool(is_rms)), int(bool(norm_only)), float(eps),
         _p(x), _p(keep[0]), _p(residual), _p(keep[1]), _p(gate), _p(keep[2]),
-        _p(weight), _p(bias), _p(scale), _p(keep[3]), _p(shift), _p(keep[4]),
+        _p(w16), _p(b16), _p(w32), _p(b32), _p(scale), _p(keep[3]), _p(shift), _p(keep[4]),
         _p(y), _p(out_st), _p(r), _p(out_st), _p(n), _p(stats))
     if rc != 0:
         raise ValueError("oracle rejected its arguments")

@@ -22,7 +22,9 @@
  *      returned; the norm acts on this rounded r.  Norm-only: r = x, nothing returned.
  *   3. LayerNorm: mu = sum(r)/D, var = sum((r - mu)^2)/D (biased, two passes),
  *      n = (r - mu) / sqrt(var + eps).   RMSNorm: ms = sum(r^2)/D, n = r / sqrt(ms + eps).
- *   4. affine: n = n * weight (if any), then n = n + bias (if any).
+ *   4. affine: n = n * weight (if any), then n = n + bias (if any). weight and bias are
+ *      bf16, or binary32 when given as float arrays (the pages' kernel takes fp32
+ *      affine parameters and casts them to bf16; here they are used as given).
  *   5. modulation: y = n * (1 + scale) + shift, rounded to bf16.
  * Every step runs in fp64 on the bf16 input values; each bf16 rounding is a single
  * round-to-nearest-even of the fp64 value (bf16_rne below, written from the IEEE
@@ -77,8 +79,10 @@ static int64_t row_offset(const int64_t* st, int64_t b, int64_t f, int64_t l) {
 /*
  * The whole op on host memory. Operand strides `*_st` are {stride_b, stride_f,
  * stride_l} in elements (0 = broadcast); output strides are {stride_b, stride_l}.
- * gate, weight, bias may be NULL (absent). norm_only != 0: residual, gate and r
- * must be NULL, and x is normalised directly.
+ * gate, weight, bias may be NULL (absent); weight_f32 / bias_f32 give the affine
+ * parameters as binary32 instead (at most one of weight / weight_f32, and of bias /
+ * bias_f32). norm_only != 0: residual, gate and r must be NULL, and x is normalised
+ * directly.
  * Optional outputs: n_out (fp64 n after the norm, before the affine step, laid out
  * like y) and stats (3 doubles per row b*L + l: mean or 0, variance or mean-square,
  * 1/sqrt(. + eps)).
@@ -90,6 +94,7 @@ int oracle_fused_norm(int64_t B, int64_t L, int64_t D, int64_t tokens_per_frame,
                       const uint16_t* res, const int64_t* res_st,
                       const uint16_t* gate, const int64_t* gate_st,
                       const uint16_t* weight, const uint16_t* bias,
+                      const float* weight_f32, const float* bias_f32,
                       const uint16_t* scale, const int64_t* scale_st,
                       const uint16_t* shift, const int64_t* shift_st,
                       uint16_t* y, const int64_t* y_st,
@@ -100,6 +105,7 @@ int oracle_fused_norm(int64_t B, int64_t L, int64_t D, int64_t tokens_per_frame,
   if (!x || !scale || !shift || !y) return -1;
   if (norm_only && (res || gate || r)) return -1;
   if (!norm_only && (!res || !r)) return -1;
+  if ((weight && weight_f32) || (bias && bias_f32)) return -1;
   int64_t rows = B * L;
   int bad = 0;
 #pragma omp parallel
@@ -158,7 +164,9 @@ int oracle_fused_norm(int64_t B, int64_t L, int64_t D, int64_t tokens_per_frame,
         double n = (v[c] - mu) * rho;
         if (n_out) n_out[b * y_st[0] + l * y_st[1] + c] = n;
         if (weight) n = n * oracle_bf16_to_double(weight[c]);
+        if (weight_f32) n = n * (double)weight_f32[c];
         if (bias) n = n + oracle_bf16_to_double(bias[c]);
+        if (bias_f32) n = n + (double)bias_f32[c];
         double yv = n * (1.0 + oracle_bf16_to_double(sr[c])) + oracle_bf16_to_double(tr[c]);
         yr[c] = oracle_bf16_rne(yv);
       }

@@ -29,7 +29,8 @@ EXPORTED = ("fused_norm_create", "fused_norm_validate", "fused_norm_launch", "fu
 class fn_config(ctypes.Structure):
     _fields_ = [("D", ctypes.c_int), ("is_rms", ctypes.c_int), ("has_gate", ctypes.c_int),
                 ("has_weight", ctypes.c_int), ("has_bias", ctypes.c_int),
-                ("norm_only", ctypes.c_int), ("eps", ctypes.c_double)]
+                ("norm_only", ctypes.c_int), ("affine_fp32", ctypes.c_int),
+                ("eps", ctypes.c_double)]
 
 
 class fn_operand(ctypes.Structure):

@@ -12,6 +12,9 @@ shapes to (pointer, strides) and makes one fused_norm_launch. Inputs must be bf1
 CUDA tensors with a contiguous channel dimension; anything else raises (there is no
 fallback path).
 
+weight and bias are (D,) vectors, bf16 or fp32 (both the same dtype when both are given);
+fp32 values are used at full precision.
+
 Accepted operand shapes for gate / scale / shift against x of shape (B, L, D):
     (D,), (1, D), (1, 1, D)      broadcast
     (B, L, D)                    per token
@@ -32,13 +35,15 @@ _handles_lock = threading.Lock()
 
 
 def _handle(D: int, is_rms: bool, has_gate: bool, has_weight: bool, has_bias: bool,
-            norm_only: bool, eps: float) -> int:
-    key = (D, is_rms, has_gate, has_weight, has_bias, norm_only, float(eps))
+            norm_only: bool, eps: float, affine_fp32: bool = False) -> int:
+    key = (D, is_rms, has_gate, has_weight, has_bias, norm_only, float(eps), affine_fp32)
     with _handles_lock:
         h = _handles.get(key)
         if h is None:
-            cfg = _abi.fn_config(D, int(is_rms), int(has_gate), int(has_weight), int(has_bias),
-                                 int(norm_only), float(eps))
+            cfg = _abi.fn_config(D=D, is_rms=int(is_rms), has_gate=int(has_gate),
+                                 has_weight=int(has_weight), has_bias=int(has_bias),
+                                 norm_only=int(norm_only), affine_fp32=int(affine_fp32),
+                                 eps=float(eps))
             st, h = _abi.fused_norm_create(cfg)
             if st != _abi.FN_OK:
                 raise _abi.FusedNormError(st, "fused_norm_create", _abi.fused_norm_status_string(st))
@@ -91,6 +96,12 @@ def _operand(t: Optional[torch.Tensor], name: str, B: int, L: int, D: int, devic
 def _vector(t: Optional[torch.Tensor], name: str, D: int, device):
     if t is None:
         return None
+    if t.dtype == torch.float32:       # fp32 affine parameters are used as given
+        if t.device != device:
+            raise ValueError(f"{name} is on {t.device}, expected {device}")
+        if t.numel() != D or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous ({D},) vector")
+        return t.data_ptr()
     _check_tensor(t, name, device)
     if t.numel() != D or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous ({D},) vector")
@@ -103,6 +114,15 @@ def _norm_flag(norm_type: str) -> bool:
     if norm_type in ("rms", "rmsnorm"):
         return True
     raise ValueError(f"norm_type must be 'layer' or 'rms', got {norm_type!r}")
+
+
+def _affine_fp32(weight, bias) -> bool:
+    dts = {t.dtype for t in (weight, bias) if t is not None}
+    if len(dts) > 1:
+        raise TypeError("weight and bias must have the same dtype")
+    if dts and dts.pop() not in (torch.bfloat16, torch.float32):
+        raise TypeError("weight and bias must be bfloat16 or float32")
+    return any(t is not None and t.dtype == torch.float32 for t in (weight, bias))
 
 
 def _launch(h: int, args: _abi.fn_args, device: torch.device, stream) -> None:
@@ -178,7 +198,7 @@ def fused_residual_norm_scale_shift(residual: torch.Tensor, x: torch.Tensor,
     r = residual_out if residual_out is not None else torch.empty_like(x, memory_format=torch.contiguous_format)
     args = build_args(x, residual, gate, weight, bias, scale, shift, y, r)
     h = _handle(x.shape[-1], _norm_flag(norm_type), gate is not None, weight is not None,
-                bias is not None, False, eps)
+                bias is not None, False, eps, _affine_fp32(weight, bias))
     _launch(h, args, x.device, stream)
     return y, r
 
@@ -193,6 +213,6 @@ def norm_scale_shift(x: torch.Tensor, weight: Optional[torch.Tensor], bias: Opti
     y = out if out is not None else torch.empty_like(x, memory_format=torch.contiguous_format)
     args = build_args(x, None, None, weight, bias, scale, shift, y, None)
     h = _handle(x.shape[-1], _norm_flag(norm_type), False, weight is not None, bias is not None,
-                True, eps)
+                True, eps, _affine_fp32(weight, bias))
     _launch(h, args, x.device, stream)
     return y

@@ -128,10 +128,11 @@ fn_status validate(const fused_norm_s* h, const fn_args* a) {
     if (!o->ptr) continue;
     if (!in_span(*o, &in[n_in++])) return FN_ERR_INVALID_ARG;
   }
+  const uintptr_t affine_bytes = (uintptr_t)D * (c.affine_fp32 ? 4 : 2);
   for (const void* v : {a->weight, a->bias}) {
     if (!v) continue;
     uintptr_t lo = reinterpret_cast<uintptr_t>(v);
-    in[n_in++] = Span{lo, lo + (uintptr_t)D * 2};
+    in[n_in++] = Span{lo, lo + affine_bytes};
   }
   int64_t ye = operand_extent(B, L, 1, D, a->y_stride_b, 0, a->y_stride_l);
   if (ye < 0) return FN_ERR_INVALID_ARG;
@@ -165,13 +166,14 @@ RowParams make_params(const fused_norm_s* h, const fn_args* a) {
   RowParams p;
   std::memset(&p, 0, sizeof(p));
   auto u16 = [](const void* v) { return static_cast<const uint16_t*>(v); };
+  auto raw = [](const void* v) { return v; };
   p.x = u16(a->x.ptr);
   p.res = u16(a->residual.ptr);
   p.gate = u16(a->gate.ptr);
   p.scale = u16(a->scale.ptr);
   p.shift = u16(a->shift.ptr);
-  p.weight = u16(a->weight);
-  p.bias = u16(a->bias);
+  p.weight = raw(a->weight);
+  p.bias = raw(a->bias);
   p.y = static_cast<uint16_t*>(a->y);
   p.r = static_cast<uint16_t*>(a->r);
   p.x_sb = a->x.stride_b; p.x_sf = a->x.stride_f; p.x_sl = a->x.stride_l;
@@ -207,13 +209,13 @@ int64_t grid_for(int64_t rows) {
 
 namespace fused_norm_impl {
 LaunchFn select_launcher(int D, bool is_rms, bool norm_only, bool has_gate, bool has_weight,
-                         bool has_bias) {
+                         bool has_bias, bool f32) {
   if (D == 5120)
-    return is_rms ? select_launcher_5120_rms(norm_only, has_gate, has_weight, has_bias)
-                  : select_launcher_5120_ln(norm_only, has_gate, has_weight, has_bias);
+    return is_rms ? select_launcher_5120_rms(norm_only, has_gate, has_weight, has_bias, f32)
+                  : select_launcher_5120_ln(norm_only, has_gate, has_weight, has_bias, f32);
   if (D == 10240)
-    return is_rms ? select_launcher_10240_rms(norm_only, has_gate, has_weight, has_bias)
-                  : select_launcher_10240_ln(norm_only, has_gate, has_weight, has_bias);
+    return is_rms ? select_launcher_10240_rms(norm_only, has_gate, has_weight, has_bias, f32)
+                  : select_launcher_10240_ln(norm_only, has_gate, has_weight, has_bias, f32);
   return nullptr;
 }
 }  // namespace fused_norm_impl
@@ -224,12 +226,14 @@ fn_status fused_norm_create(fused_norm_t* out, const fn_config* cfg) {
   if (!out || !cfg) return FN_ERR_INVALID_ARG;
   const fn_config& c = *cfg;
   if (!is_flag(c.is_rms) || !is_flag(c.has_gate) || !is_flag(c.has_weight) ||
-      !is_flag(c.has_bias) || !is_flag(c.norm_only))
+      !is_flag(c.has_bias) || !is_flag(c.norm_only) || !is_flag(c.affine_fp32))
     return FN_ERR_INVALID_ARG;
+  if (c.affine_fp32 && !c.has_weight && !c.has_bias) return FN_ERR_INVALID_ARG;
   if (!std::isfinite(c.eps) || c.eps < 0.0) return FN_ERR_INVALID_ARG;
   if (c.norm_only && c.has_gate) return FN_ERR_INVALID_ARG;
   if (c.D != 5120 && c.D != 10240) return FN_ERR_UNSUPPORTED;
-  LaunchFn fn = select_launcher(c.D, c.is_rms, c.norm_only, c.has_gate, c.has_weight, c.has_bias);
+  LaunchFn fn = select_launcher(c.D, c.is_rms, c.norm_only, c.has_gate, c.has_weight, c.has_bias,
+                                c.affine_fp32);
   if (!fn) return FN_ERR_UNSUPPORTED;
   fused_norm_s* h = new (std::nothrow) fused_norm_s;
   if (!h) return FN_ERR_INVALID_ARG;

@@ -46,8 +46,8 @@ struct RowParams {
   const uint16_t* gate;
   const uint16_t* scale;
   const uint16_t* shift;
-  const uint16_t* weight;
-  const uint16_t* bias;
+  const void* weight;  // (D) bf16, or fp32 when AFFINE_F32
+  const void* bias;
   uint16_t* y;
   uint16_t* r;
   int64_t x_sb, x_sf, x_sl;
@@ -183,13 +183,11 @@ __device__ __forceinline__ uint32_t y_exact(float v, float w, float b, float s, 
 // lies in the lowest interval of a binade, one at least ulp/4 below (ulp = bf16 spacing
 // at y; |y| 2^-10 <= ulp/4). So y rounds correctly if B < min(D, |y| 2^-10).
 template <int H, bool HAS_WEIGHT, bool HAS_BIAS>
-__device__ __forceinline__ float y_fast(uint32_t vw, uint32_t sw, uint32_t tw, uint32_t ww,
-                                        uint32_t bw, const RowStats& st, bool& near) {
+__device__ __forceinline__ float y_fast_core(uint32_t vw, uint32_t sw, uint32_t tw, float w, float b,
+                                             const RowStats& st, bool& near) {
   constexpr float k8u = 4.76837158203125e-7f;  // 2^-21
   const float n = add_bf16_f32<H>(vw, st.neg_mu32) * st.rho32;
-  const float w = H ? hi_f(ww) : lo_f(ww);
   const float nw = HAS_WEIGHT ? n * w : n;
-  const float b = H ? hi_f(bw) : lo_f(bw);
   const float nb = HAS_BIAS ? nw + b : nw;
   const float a = add_bf16_f32<H>(sw, 1.0f);
   const float t = H ? hi_f(tw) : lo_f(tw);
@@ -202,6 +200,14 @@ __device__ __forceinline__ float y_fast(uint32_t vw, uint32_t sw, uint32_t tw, u
   const float room = fminf(fabsf(y - mid), fabsf(y) * 9.765625e-4f);  // 2^-10
   near |= !(room > bound);  // NaN/Inf also take the fp64 path
   return y;
+}
+
+// y_fast_core with bf16 weight / bias taken from packed words.
+template <int H, bool HAS_WEIGHT, bool HAS_BIAS>
+__device__ __forceinline__ float y_fast(uint32_t vw, uint32_t sw, uint32_t tw, uint32_t ww,
+                                        uint32_t bw, const RowStats& st, bool& near) {
+  return y_fast_core<H, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, H ? hi_f(ww) : lo_f(ww),
+                                              H ? hi_f(bw) : lo_f(bw), st, near);
 }
 
 // Element q's value from a 16-byte vector, for a runtime q (rare paths only).
@@ -236,6 +242,55 @@ __device__ __forceinline__ uint4 output_vec(const uint4& v, const uint4& sv, con
     const uint32_t bits = y_exact<HAS_WEIGHT, HAS_BIAS>(
         elem_dyn(v, q), HAS_WEIGHT ? elem_dyn(wv, q) : 1.0f, HAS_BIAS ? elem_dyn(bv, q) : 0.0f,
         elem_dyn(sv, q), elem_dyn(tv, q), st.mu, st.rho);
+    const uint32_t put = (q & 1) ? (bits << 16) : bits;
+    const uint32_t keep = (q & 1) ? 0x0000FFFFu : 0xFFFF0000u;
+    const int i = q >> 1;
+    out.x = i == 0 ? ((out.x & keep) | put) : out.x;
+    out.y = i == 1 ? ((out.y & keep) | put) : out.y;
+    out.z = i == 2 ? ((out.z & keep) | put) : out.z;
+    out.w = i == 3 ? ((out.w & keep) | put) : out.w;
+  }
+  return out;
+}
+
+// fp32 affine parameters (w, b as given, 8 per vector: two 16-byte loads each).
+struct Affine8 {
+  float v[8];
+};
+__device__ __forceinline__ Affine8 load_affine_f32(const void* p, int j) {
+  const float4* f = reinterpret_cast<const float4*>(p) + 2 * j;
+  const float4 a = __ldg(f), c = __ldg(f + 1);
+  return Affine8{{a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w}};
+}
+__device__ __forceinline__ float sel8(const Affine8& a, int q) {
+  return q == 0 ? a.v[0] : q == 1 ? a.v[1] : q == 2 ? a.v[2] : q == 3 ? a.v[3]
+       : q == 4 ? a.v[4] : q == 5 ? a.v[5] : q == 6 ? a.v[6] : a.v[7];
+}
+
+// As output_vec, with fp32 weight / bias.
+template <bool HAS_WEIGHT, bool HAS_BIAS>
+__device__ __forceinline__ uint4 output_vec_f32(const uint4& v, const uint4& sv, const uint4& tv,
+                                                const Affine8& wf, const Affine8& bf,
+                                                const RowStats& st) {
+  uint32_t o[4];
+  uint32_t near_mask = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t vw = word(v, i), sw = word(sv, i), tw = word(tv, i);
+    bool n0 = false, n1 = false;
+    const float y0 = y_fast_core<0, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, wf.v[2 * i], bf.v[2 * i], st, n0);
+    const float y1 = y_fast_core<1, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, wf.v[2 * i + 1], bf.v[2 * i + 1], st, n1);
+    o[i] = pack_rn(y0, y1);
+    near_mask |= (n0 ? 1u : 0u) << (2 * i);
+    near_mask |= (n1 ? 2u : 0u) << (2 * i);
+  }
+  uint4 out = make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll 1
+  while (near_mask) {  // rare
+    const int q = __ffs(near_mask) - 1;
+    near_mask &= near_mask - 1;
+    const uint32_t bits = y_exact<HAS_WEIGHT, HAS_BIAS>(elem_dyn(v, q), sel8(wf, q), sel8(bf, q),
+                                                        elem_dyn(sv, q), elem_dyn(tv, q), st.mu, st.rho);
     const uint32_t put = (q & 1) ? (bits << 16) : bits;
     const uint32_t keep = (q & 1) ? 0x0000FFFFu : 0xFFFF0000u;
     const int i = q >> 1;
@@ -282,7 +337,8 @@ struct MinBlocks {
           ? 4 : RowShape<D>::kMinBlocks;
 };
 
-template <int D, int VPT, bool IS_RMS, bool NORM_ONLY, bool HAS_GATE, bool HAS_WEIGHT, bool HAS_BIAS>
+template <int D, int VPT, bool IS_RMS, bool NORM_ONLY, bool HAS_GATE, bool HAS_WEIGHT, bool HAS_BIAS,
+          bool AFFINE_F32>
 __global__ void __launch_bounds__(D / (8 * VPT), (MinBlocks<D, IS_RMS, HAS_WEIGHT, HAS_BIAS>::value))
 fused_norm_rows(const RowParams p) {
   constexpr int T = D / (8 * VPT);
@@ -423,56 +479,67 @@ fused_norm_rows(const RowParams p) {
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
       const int j = tid + k * T;
-      uint4 wv = make_uint4(0, 0, 0, 0), bv = make_uint4(0, 0, 0, 0);
-      if (HAS_WEIGHT) wv = __ldg(reinterpret_cast<const uint4*>(p.weight) + j);
-      if (HAS_BIAS) bv = __ldg(reinterpret_cast<const uint4*>(p.bias) + j);
-      __stcs(yo + j, output_vec<HAS_WEIGHT, HAS_BIAS>(v[k], sv[k], tv[k], wv, bv, st));
+      if (AFFINE_F32) {
+        Affine8 wf{{1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f}}, bf{{0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}};
+        if (HAS_WEIGHT) wf = load_affine_f32(p.weight, j);
+        if (HAS_BIAS) bf = load_affine_f32(p.bias, j);
+        __stcs(yo + j, output_vec_f32<HAS_WEIGHT, HAS_BIAS>(v[k], sv[k], tv[k], wf, bf, st));
+      } else {
+        uint4 wv = make_uint4(0, 0, 0, 0), bv = make_uint4(0, 0, 0, 0);
+        if (HAS_WEIGHT) wv = __ldg(reinterpret_cast<const uint4*>(p.weight) + j);
+        if (HAS_BIAS) bv = __ldg(reinterpret_cast<const uint4*>(p.bias) + j);
+        __stcs(yo + j, output_vec<HAS_WEIGHT, HAS_BIAS>(v[k], sv[k], tv[k], wv, bv, st));
+      }
     }
   }
 }
 
-template <int D, int VPT, bool IS_RMS, bool NORM_ONLY, bool HAS_GATE, bool HAS_WEIGHT, bool HAS_BIAS>
+template <int D, int VPT, bool IS_RMS, bool NORM_ONLY, bool HAS_GATE, bool HAS_WEIGHT, bool HAS_BIAS,
+          bool AFFINE_F32>
 cudaError_t launch_rows(const RowParams& p, int64_t grid, cudaStream_t stream) {
   constexpr int T = D / (8 * VPT);
-  fused_norm_rows<D, VPT, IS_RMS, NORM_ONLY, HAS_GATE, HAS_WEIGHT, HAS_BIAS>
+  fused_norm_rows<D, VPT, IS_RMS, NORM_ONLY, HAS_GATE, HAS_WEIGHT, HAS_BIAS, AFFINE_F32>
       <<<(unsigned)grid, T, 0, stream>>>(p);
   return cudaGetLastError();
 }
 
-// Launcher for a specialisation, selected at create time. Defined in one
-// translation unit per (D, norm type) so the instances compile in parallel.
+// Launcher for one (norm_only, gate) group: the affine combinations.
+template <int D, bool RMS, bool NO, bool G>
+LaunchFn pick_affine(bool w, bool b, bool f32) {
+  constexpr int V = RowShape<D>::VPT;
+  if (!w && !b) return &launch_rows<D, V, RMS, NO, G, false, false, false>;
+  if (f32) {
+    if (w && b) return &launch_rows<D, V, RMS, NO, G, true, true, true>;
+    return w ? &launch_rows<D, V, RMS, NO, G, true, false, true>
+             : &launch_rows<D, V, RMS, NO, G, false, true, true>;
+  }
+  if (w && b) return &launch_rows<D, V, RMS, NO, G, true, true, false>;
+  return w ? &launch_rows<D, V, RMS, NO, G, true, false, false>
+           : &launch_rows<D, V, RMS, NO, G, false, true, false>;
+}
+
+// Launcher for every specialisation of one (D, norm); instantiated in one translation
+// unit per (D, norm) so the instances compile in parallel.
+template <int D, bool RMS>
+LaunchFn pick_launcher(bool norm_only, bool has_gate, bool has_weight, bool has_bias, bool f32) {
+  if (norm_only) return pick_affine<D, RMS, true, false>(has_weight, has_bias, f32);
+  return has_gate ? pick_affine<D, RMS, false, true>(has_weight, has_bias, f32)
+                  : pick_affine<D, RMS, false, false>(has_weight, has_bias, f32);
+}
+
 LaunchFn select_launcher(int D, bool is_rms, bool norm_only, bool has_gate, bool has_weight,
-                         bool has_bias);
-LaunchFn select_launcher_5120_ln(bool norm_only, bool has_gate, bool has_weight, bool has_bias);
-LaunchFn select_launcher_5120_rms(bool norm_only, bool has_gate, bool has_weight, bool has_bias);
-LaunchFn select_launcher_10240_ln(bool norm_only, bool has_gate, bool has_weight, bool has_bias);
-LaunchFn select_launcher_10240_rms(bool norm_only, bool has_gate, bool has_weight, bool has_bias);
+                         bool has_bias, bool affine_f32);
+LaunchFn select_launcher_5120_ln(bool norm_only, bool has_gate, bool has_weight, bool has_bias, bool f32);
+LaunchFn select_launcher_5120_rms(bool norm_only, bool has_gate, bool has_weight, bool has_bias, bool f32);
+LaunchFn select_launcher_10240_ln(bool norm_only, bool has_gate, bool has_weight, bool has_bias, bool f32);
+LaunchFn select_launcher_10240_rms(bool norm_only, bool has_gate, bool has_weight, bool has_bias, bool f32);
 
 }  // namespace fused_norm_impl
 
-// Instantiates the 12 (norm_only, gate, weight, bias) launchers for one (D, norm).
+// Defines the launcher selector of one (D, norm) translation unit.
 #define FUSED_NORM_DEFINE_SELECTOR(NAME, D_, RMS_)                                              \
   namespace fused_norm_impl {                                                                   \
-  LaunchFn NAME(bool norm_only, bool has_gate, bool has_weight, bool has_bias) {                \
-    constexpr int V = RowShape<D_>::VPT;                                                        \
-    if (norm_only) {                                                                            \
-      if (has_weight)                                                                           \
-        return has_bias ? &launch_rows<D_, V, RMS_, true, false, true, true>                    \
-                        : &launch_rows<D_, V, RMS_, true, false, true, false>;                  \
-      return has_bias ? &launch_rows<D_, V, RMS_, true, false, false, true>                     \
-                      : &launch_rows<D_, V, RMS_, true, false, false, false>;                   \
-    }                                                                                           \
-    if (has_gate) {                                                                             \
-      if (has_weight)                                                                           \
-        return has_bias ? &launch_rows<D_, V, RMS_, false, true, true, true>                    \
-                        : &launch_rows<D_, V, RMS_, false, true, true, false>;                  \
-      return has_bias ? &launch_rows<D_, V, RMS_, false, true, false, true>                     \
-                      : &launch_rows<D_, V, RMS_, false, true, false, false>;                   \
-    }                                                                                           \
-    if (has_weight)                                                                             \
-      return has_bias ? &launch_rows<D_, V, RMS_, false, false, true, true>                     \
-                      : &launch_rows<D_, V, RMS_, false, false, true, false>;                   \
-    return has_bias ? &launch_rows<D_, V, RMS_, false, false, false, true>                      \
-                    : &launch_rows<D_, V, RMS_, false, false, false, false>;                    \
+  LaunchFn NAME(bool norm_only, bool has_gate, bool has_weight, bool has_bias, bool f32) {      \
+    return pick_launcher<D_, RMS_>(norm_only, has_gate, has_weight, has_bias, f32);             \
   }                                                                                             \
   }

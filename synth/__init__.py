@@ -53,6 +53,8 @@ def _load():
     lib.synth_fill_bf16_rows.restype = None
     lib.synth_value_bf16.argtypes = [i64, i64, u64, u32, dbl, dbl, dbl]
     lib.synth_value_bf16.restype = ctypes.c_uint16
+    lib.synth_fill_f32_row.argtypes = [vp, i64, u64, u32, dbl, dbl]
+    lib.synth_fill_f32_row.restype = None
     lib.synth_pick_rows.argtypes = [i64, i64, u64, vp, vp]
     lib.synth_pick_rows.restype = None
     _lib = lib
@@ -233,6 +235,15 @@ class Workload:
             out = np.empty((len(rows), self.D), dtype=np.uint16)
         mult = self.row_mult(rows) if tensor in ("x", "residual") else None
         return fill_rows(out, rows, self.seed, tensor, mu, sigma, mult)
+
+    def generate_f32(self, tensor: str) -> np.ndarray:
+        """A (D,) float32 affine parameter (weight or bias): the same draws as generate(),
+        kept at binary32 precision."""
+        assert tensor in ("weight", "bias")
+        mu, sigma = self.dist(tensor)
+        out = np.empty(self.D, dtype=np.float32)
+        _load().synth_fill_f32_row(_ptr(out), self.D, self.seed, TENSOR_IDS[tensor], mu, sigma)
+        return out
 
     def token_rows(self, operand: str, flat_rows: np.ndarray) -> np.ndarray:
         """Stored rows of `operand` read by the given flattened tokens b*L + l."""

@@ -103,6 +103,14 @@ void synth_fill_bf16_rows(uint16_t* out, int64_t pitch, const int64_t* rows, int
   }
 }
 
+/* Like synth_fill_bf16 for one (1, D) row, but the values are kept as binary32 (the
+ * same draws, rounded to float only). For fp32 affine parameters. */
+void synth_fill_f32_row(float* out, int64_t D, uint64_t seed, uint32_t tensor_id, double mu,
+                        double sigma) {
+  uint64_t k = stream_key(seed, tensor_id, 0);
+  for (int64_t c = 0; c < D; ++c) out[c] = (float)(mu + sigma * normal_at(k, c));
+}
+
 /* Single element, for spot checks of the fill above. */
 uint16_t synth_value_bf16(int64_t row, int64_t c, uint64_t seed, uint32_t tensor_id, double mu,
                           double sigma, double mult) {

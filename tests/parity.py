@@ -106,8 +106,10 @@ def oracle_rows(w: synth.Workload, spec: synth.Spec, host, flat_rows: np.ndarray
         res_st=None if spec.norm_only else st,
         gate=pick("gate") if (spec.has_gate and not spec.norm_only) else None,
         gate_st=st if (spec.has_gate and not spec.norm_only) else None,
-        weight=host["weight"] if spec.has_weight else None,
-        bias=host["bias"] if spec.has_bias else None,
+        weight=(host["weight"].reshape(-1) if host["weight"].dtype == np.float32 else host["weight"])
+        if spec.has_weight else None,
+        bias=(host["bias"].reshape(-1) if host["bias"].dtype == np.float32 else host["bias"])
+        if spec.has_bias else None,
         scale=pick("scale"), scale_st=st, shift=pick("shift"), shift_st=st,
         is_rms=spec.is_rms, norm_only=spec.norm_only, eps=w.eps)
 

@@ -54,8 +54,13 @@ def test_struct_layouts_match_header():
     assert [int(v) for v in got] == want
 
 
-def make(D=5120, is_rms=0, gate=1, weight=0, bias=0, norm_only=0, eps=1e-6):
-    st, h = fn.fused_norm_create(fn.fn_config(D, is_rms, gate, weight, bias, norm_only, eps))
+def cfg(D=5120, is_rms=0, gate=1, weight=0, bias=0, norm_only=0, eps=1e-6, affine_fp32=0):
+    return fn.fn_config(D=D, is_rms=is_rms, has_gate=gate, has_weight=weight, has_bias=bias,
+                        norm_only=norm_only, affine_fp32=affine_fp32, eps=eps)
+
+
+def make(D=5120, is_rms=0, gate=1, weight=0, bias=0, norm_only=0, eps=1e-6, affine_fp32=0):
+    st, h = fn.fused_norm_create(cfg(D, is_rms, gate, weight, bias, norm_only, eps, affine_fp32))
     assert st == OK
     return h
 
@@ -92,28 +97,30 @@ def valid_args(B=2, L=8, D=5120, gate=True, weight=False, bias=False, norm_only=
 
 @pytest.mark.parametrize("D,want", [(5120, OK), (10240, OK), (4096, UNS), (5128, UNS), (0, UNS), (-5120, UNS)])
 def test_create_D(D, want):
-    st, h = fn.fused_norm_create(fn.fn_config(D, 0, 1, 0, 0, 0, 1e-6))
+    st, h = fn.fused_norm_create(cfg(D=D))
     assert st == want
     if h:
         fn.fused_norm_destroy(h)
 
 
-@pytest.mark.parametrize("cfg", [
+@pytest.mark.parametrize("args", [
     (5120, 2, 1, 0, 0, 0, 1e-6), (5120, 0, -1, 0, 0, 0, 1e-6), (5120, 0, 1, 3, 0, 0, 1e-6),
     (5120, 0, 1, 0, 0, 1, 1e-6),            # norm-only with a gate
     (5120, 0, 1, 0, 0, 0, -1e-6), (5120, 0, 1, 0, 0, 0, float("nan")), (5120, 0, 1, 0, 0, 0, float("inf")),
+    (5120, 0, 1, 0, 0, 0, 1e-6, 1),         # fp32 affine without weight or bias
+    (5120, 0, 1, 1, 0, 0, 1e-6, 2),         # affine_fp32 not a flag
 ])
-def test_create_rejects(cfg):
-    st, h = fn.fused_norm_create(fn.fn_config(*cfg))
+def test_create_rejects(args):
+    st, h = fn.fused_norm_create(cfg(*args))
     assert st == INV and h is None
 
 
 def test_create_null_and_config_roundtrip():
     assert fn.load().fused_norm_create(None, None) == INV
-    h = make(D=10240, is_rms=1, gate=0, weight=1, bias=1)
-    st, cfg = fn.fused_norm_get_config(h)
-    assert st == OK and (cfg.D, cfg.is_rms, cfg.has_gate, cfg.has_weight, cfg.has_bias) == (10240, 1, 0, 1, 1)
-    assert abs(cfg.eps - 1e-6) < 1e-12
+    h = make(D=10240, is_rms=1, gate=0, weight=1, bias=1, affine_fp32=1)
+    st, c = fn.fused_norm_get_config(h)
+    assert st == OK and (c.D, c.is_rms, c.has_gate, c.has_weight, c.has_bias, c.affine_fp32) == (10240, 1, 0, 1, 1, 1)
+    assert c.eps == 1e-6
     assert fn.fused_norm_destroy(h) == OK
     assert fn.fused_norm_destroy(None) == OK
 
@@ -232,3 +239,13 @@ def test_null_handle_and_args():
     assert fn.load().fused_norm_validate(None, None) == INV
     h = make()
     assert fn.load().fused_norm_validate(h, None) == INV
+
+
+def test_fp32_affine_extent_in_overlap_rules():
+    # fp32 weight spans 4*D bytes: y placed right after a bf16-sized weight overlaps it
+    h16, h32 = make(weight=1), make(weight=1, affine_fp32=1)
+    a = valid_args(weight=True)
+    a.y = a.weight + 5120 * 2
+    a.y_stride_b, a.y_stride_l = 8 * 5120, 5120
+    assert fn.fused_norm_validate(h16, a) == OK
+    assert fn.fused_norm_validate(h32, a) == INV

@@ -11,6 +11,7 @@ import numpy as np
 import pytest
 import torch
 
+import rmsnorm_row_b200 as fn
 import synth
 from parity import Tally, check_workload, host_inputs, run_gpu, upload_host
 
@@ -108,3 +109,43 @@ def test_frame_gate_B1_F21x8400_full():
 
 def test_frame_gate_B1_F49x3600_full():
     _full_size(synth.W5B)
+
+
+# ---- fp32 affine parameters ----------------------------------------------------------
+
+@pytest.mark.parametrize("D", [5120, 10240])
+@pytest.mark.parametrize("spec", [synth.Spec(False, True, True, has_bias=True),
+                                  synth.Spec(True, False, True),
+                                  synth.Spec(False, False, False, has_bias=True),
+                                  synth.Spec(True, False, True, has_bias=True, norm_only=True)],
+                         ids=lambda s: s.name)
+def test_fp32_affine(D, spec):
+    # weight and bias as fp32 (the same draws as the bf16 ones, kept at 24 bits), used at
+    # full precision on both sides
+    import oracle
+    from parity import oracle_rows
+    base = synth.W3 if D == 5120 else synth.W3B
+    w = synth.scaled(base, 613)
+    host = host_inputs(w)
+    dev = upload_host(w, host, DEV)
+    w32 = torch.from_numpy(w.generate_f32("weight")).to(DEV) if spec.has_weight else None
+    b32 = torch.from_numpy(w.generate_f32("bias")).to(DEV) if spec.has_bias else None
+    norm = "rms" if spec.is_rms else "layer"
+    if spec.norm_only:
+        y, r = fn.norm_scale_shift(dev["x"], w32, b32, dev["scale"], dev["shift"], norm, w.eps), None
+    else:
+        y, r = fn.fused_residual_norm_scale_shift(dev["residual"], dev["x"],
+                                                  dev["gate"] if spec.has_gate else None, w32, b32,
+                                                  dev["scale"], dev["shift"], norm, w.eps)
+    torch.cuda.synchronize()
+    host32 = dict(host)
+    host32["weight"] = w.generate_f32("weight")
+    host32["bias"] = w.generate_f32("bias")
+    ref = oracle_rows(w, spec, host32, np.arange(w.rows))
+    from synth.device import to_bits
+    ty, tr = Tally(), Tally()
+    ty.add(to_bits(y).reshape(-1, D), ref["y"][0])
+    if r is not None:
+        tr.add(to_bits(r).reshape(-1, D), ref["r"][0])
+    _assert(ty, tr, f"{w.name}/{spec.name}/fp32-affine")
+    assert ty.exact == ty.n

@@ -29,6 +29,8 @@ MUTANTS = [
     ("modulation_without_one", "n * (1.0 + oracle_bf16_to_double(sr[c]))", "n * (oracle_bf16_to_double(sr[c]))", 0),
     ("weight_added", "n = n * oracle_bf16_to_double(weight[c]);", "n = n + oracle_bf16_to_double(weight[c]);", 0),
     ("bias_dropped", "n = n + oracle_bf16_to_double(bias[c]);", "n = n;", 0),
+    ("fp32_weight_cast_to_bf16", "if (weight_f32) n = n * (double)weight_f32[c];",
+     "if (weight_f32) n = n * oracle_bf16_to_double(oracle_bf16_rne((double)weight_f32[c]));", 0),
     ("frame_index_mod", "l / tokens_per_frame : 0", "l % tokens_per_frame : 0", 0),
     ("ties_away", "(frac == 0.5 && fmod(whole, 2.0) == 1.0)", "(frac == 0.5)", 0),
     ("rounding_truncates", "if (frac > 0.5 || (frac == 0.5 && fmod(whole, 2.0) == 1.0)) whole += 1.0;", "", 0),

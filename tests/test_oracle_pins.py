@@ -424,3 +424,41 @@ def test_oracle_rejects_bad_arguments():
     with pytest.raises(ValueError):
         oracle.fused_norm(1, 3, D, x=a, x_st=st, residual=a, res_st=st, scale=a, scale_st=st,
                           shift=a, shift_st=st, tokens_per_frame=2)
+
+
+# --------------------------------------------------------------------------
+# fp32 affine parameters (used as given, not cast to bf16)
+# --------------------------------------------------------------------------
+
+def test_fp32_affine_equal_to_bf16_when_representable():
+    D = 64
+    rng = np.random.default_rng(12)
+    r, s, t = _rand_bf16(rng, D), _rand_bf16(rng, D, 0, .1), _rand_bf16(rng, D, 0, .1)
+    wt, bs = _rand_bf16(rng, D, 1, .1), _rand_bf16(rng, D, 0, .1)   # bf16-exact values
+    a = one_row(r, scale=s, shift=t, weight=wt, bias=bs)
+    st = (D, 0, D)
+    b = oracle.fused_norm(1, 1, D, x=exact_bits(np.zeros(D)), x_st=st, residual=exact_bits(r), res_st=st,
+                          weight=wt.astype(np.float32), bias=bs.astype(np.float32),
+                          scale=exact_bits(s), scale_st=st, shift=exact_bits(t), shift_st=st, eps=EPS)
+    assert np.array_equal(a["y"], b["y"])
+
+
+def test_fp32_affine_against_exact_rationals():
+    D = 48
+    rng = np.random.default_rng(13)
+    r, s, t = _rand_bf16(rng, D), _rand_bf16(rng, D, 0, .1), _rand_bf16(rng, D, 0, .1)
+    wt = (1 + 0.1 * rng.normal(size=D)).astype(np.float32)          # 24-bit values
+    bs = (0.1 * rng.normal(size=D)).astype(np.float32)
+    st = (D, 0, D)
+    out = oracle.fused_norm(1, 1, D, x=exact_bits(np.zeros(D)), x_st=st, residual=exact_bits(r),
+                            res_st=st, weight=wt, bias=bs, scale=exact_bits(s), scale_st=st,
+                            shift=exact_bits(t), shift_st=st, eps=EPS, want_n=True)
+    n = out["n"][0, 0]
+    nonexact = 0
+    for i in range(D):
+        want = (Fraction(n[i]) * Fraction(float(wt[i])) + Fraction(float(bs[i]))) * (1 + Fraction(s[i])) + Fraction(t[i])
+        if not nearest_bf16_ok(want, int(out["y"][0, 0, i])):
+            nonexact += 1
+    assert nonexact == 0
+    # and the fp32 values really carry more than bf16 precision here
+    assert not np.array_equal(bf16_bits_to_f64(f32_to_bf16_bits_rne(wt)), wt.astype(np.float64))

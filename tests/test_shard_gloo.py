@@ -108,7 +108,7 @@ def _one_layout(rank, world, layout, B, L, D, F, q):
         import synth
         Dk = 5120
         st_k = synth.layout_strides(layout, B, L, Dk, F)
-        _, h = fn.fused_norm_create(fn.fn_config(Dk, 0, 1, 1, 0, 0, 1e-6))
+        _, h = fn.fused_norm_create(fn.fn_config(D=Dk, has_gate=1, has_weight=1, eps=1e-6))
         ok_valid = fn.fused_norm_validate(h, shard_args(_args_for(B, L, Dk, F, st_k, bases),
                                                         world, rank)) == fn.FN_OK
         part = _run_oracle_on(mine, bufs, bases, D)
