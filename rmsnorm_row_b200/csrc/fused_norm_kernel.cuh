@@ -303,7 +303,8 @@ __device__ __forceinline__ uint4 output_vec_f32(const uint4& v, const uint4& sv,
 }
 
 // Launch shape per D: vectors per thread (threads = D / (8 VPT)) and the CTAs per SM
-// the register budget is sized for (65536 / (threads * kMinBlocks) registers each).
+// the register budget is sized for (65536 / (threads * kMinBlocks) registers each),
+// the same for every specialisation of a D (measured on B200 across all of them).
 template <int D> struct RowShape;
 #ifndef FN_VPT_5120
 #define FN_VPT_5120 5
@@ -326,20 +327,9 @@ template <int D> struct RowShape;
 template <> struct RowShape<5120> { static constexpr int VPT = FN_VPT_5120, kMinBlocks = FN_MINB_5120; };
 template <> struct RowShape<10240> { static constexpr int VPT = FN_VPT_10240, kMinBlocks = FN_MINB_10240; };
 
-// CTAs per SM the register budget targets for one specialisation. D = 5120 LayerNorm
-// with an affine weight or bias needs more registers than 5 CTAs allow without spills;
-// measured on B200 (L = 90000 and the frame-gate shape), 4 CTAs is faster there, while
-// every other D = 5120 specialisation is faster at 5.
-template <int D, bool IS_RMS, bool HAS_WEIGHT, bool HAS_BIAS>
-struct MinBlocks {
-  static constexpr int value =
-      (D == 5120 && !IS_RMS && (HAS_WEIGHT || HAS_BIAS) && RowShape<D>::kMinBlocks > 4)
-          ? 4 : RowShape<D>::kMinBlocks;
-};
-
 template <int D, int VPT, bool IS_RMS, bool NORM_ONLY, bool HAS_GATE, bool HAS_WEIGHT, bool HAS_BIAS,
           bool AFFINE_F32>
-__global__ void __launch_bounds__(D / (8 * VPT), (MinBlocks<D, IS_RMS, HAS_WEIGHT, HAS_BIAS>::value))
+__global__ void __launch_bounds__(D / (8 * VPT), RowShape<D>::kMinBlocks)
 fused_norm_rows(const RowParams p) {
   constexpr int T = D / (8 * VPT);
   constexpr int W = T / 32;
@@ -447,16 +437,23 @@ fused_norm_rows(const RowParams p) {
       double var = fmax(div_by_row_length<D>(t2) - mu * mu, 0.0);
       if (mu * mu > 1048576.0 * var && var > 0.0) {
         // The mean dwarfs the spread: take the variance around the mean instead
-        // (uniform branch: every thread of the CTA has the same statistics).
+        // (uniform branch: every thread of the CTA has the same statistics). The row
+        // is read back from memory (this thread's own r stores, or x) in a rolled
+        // loop: unrolled over the register copy, this rare pass would set the
+        // kernel's register allocation and force spills on the common path.
+        const uint4* rowv = NORM_ONLY ? reinterpret_cast<const uint4*>(xr)
+                                      : reinterpret_cast<const uint4*>(p.r + (b * p.r_sb + l * p.r_sl));
         double c2 = 0.0;
-#pragma unroll
-        for (int k = 0; k < VPT; ++k)
+#pragma unroll 1
+        for (int k = 0; k < VPT; ++k) {
+          const uint4 vk = __ldcg(rowv + tid + k * T);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const double a = bf16_f64<0>(word(v[k], i)) - mu, c = bf16_f64<1>(word(v[k], i)) - mu;
+            const double a = bf16_f64<0>(word(vk, i)) - mu, c = bf16_f64<1>(word(vk, i)) - mu;
             c2 = fma(a, a, c2);
             c2 = fma(c, c, c2);
           }
+        }
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) c2 += __shfl_xor_sync(0xFFFFFFFFu, c2, o);
         if (lane == 0) centred[warp] = c2;
