@@ -61,6 +61,9 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--flush-l2", action="store_true",
+                   help="write a 512 MB buffer before every timed launch and time each launch "
+                        "alone (for the small shapes, whose inputs otherwise stay in L2)")
     p.add_argument("--graph", action="store_true",
                    help="replay the timed launches from one CUDA graph (removes host launch "
                         "overhead; for the launch-bound small shapes)")
@@ -214,7 +217,8 @@ def run_ours(args):
     host = {}
     for name in ("x", "residual", "gate", "scale", "shift", "weight", "bias"):
         if name == "gate" and not spec.has_gate or name == "weight" and not spec.has_weight \
-                or name == "bias" and not spec.has_bias:
+                or name == "bias" and not spec.has_bias \
+                or name in ("residual", "gate") and spec.norm_only:
             continue
         n = 1 if name in ("weight", "bias") else w.stored_rows(name)
         t = torch.empty((n, w.D), dtype=torch.int16, pin_memory=True)
@@ -222,13 +226,13 @@ def run_ours(args):
         host[name] = t.view(torch.bfloat16).view(synth.device.operand_view_shape(w, name))
     d = {k: v.to(dev) for k, v in host.items()}
     y = torch.empty((w.B, w.L, w.D), dtype=torch.bfloat16, device=dev)
-    r = torch.empty_like(y)
+    r = None if spec.norm_only else torch.empty_like(y)
     stream = torch.cuda.current_stream(dev)
 
     # The C arguments are marshalled once; each step is one fused_norm_launch call
     # (the tensor-level API marshals the same arguments on every call, which costs
     # ~15 us of host time and dominates the launch-bound small shapes).
-    args_c = fn.build_args(d["x"], d["residual"], d.get("gate"), d.get("weight"), d.get("bias"),
+    args_c = fn.build_args(d["x"], d.get("residual"), d.get("gate"), d.get("weight"), d.get("bias"),
                            d["scale"], d["shift"], y, r)
     handle = fn.api._handle(w.D, spec.is_rms, spec.has_gate, spec.has_weight, spec.has_bias,
                             spec.norm_only, w.eps, False)
@@ -239,9 +243,13 @@ def run_ours(args):
             raise fn.FusedNormError(st, "fused_norm_launch", fn.fused_norm_status_string(st))
 
     # one call through the tensor-level API first: same result as the prebuilt launch
-    fn.fused_residual_norm_scale_shift(d["residual"], d["x"], d.get("gate"), d.get("weight"),
-                                       d.get("bias"), d["scale"], d["shift"], norm, w.eps,
-                                       out=y, residual_out=r, stream=stream)
+    if spec.norm_only:
+        fn.norm_scale_shift(d["x"], d.get("weight"), d.get("bias"), d["scale"], d["shift"], norm,
+                            w.eps, out=y, stream=stream)
+    else:
+        fn.fused_residual_norm_scale_shift(d["residual"], d["x"], d.get("gate"), d.get("weight"),
+                                           d.get("bias"), d["scale"], d["shift"], norm, w.eps,
+                                           out=y, residual_out=r, stream=stream)
 
     def barrier():
         if world > 1:
@@ -278,6 +286,10 @@ def run_ours(args):
         torch.cuda.synchronize(dev)
         graph.replay()
         torch.cuda.synchronize(dev)
+    if args.flush_l2 and graph is not None:
+        raise SystemExit("--flush-l2 and --graph are exclusive")
+    scratch = torch.empty(128 << 20, dtype=torch.int32, device=dev) if args.flush_l2 else None
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if args.flush_l2 else None
     barrier()
     torch.cuda.synchronize(dev)
     ev[0].record(stream)
@@ -286,6 +298,13 @@ def run_ours(args):
             graph.replay()
         launches = K
         ev[K].record(stream)
+    elif scratch is not None:
+        for i in range(K):
+            scratch.zero_()           # 512 MB written: the inputs leave the 126 MB L2
+            starts[i].record(stream)
+            step()
+            launches += 1
+            ev[i + 1].record(stream)
     else:
         for i in range(K):
             step()
@@ -294,9 +313,13 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     barrier()
     clocks = sampler.stop() if sampler else None
-    per = ([ev[0].elapsed_time(ev[K]) / K] * K if graph is not None
-           else [ev[i].elapsed_time(ev[i + 1]) for i in range(K)])
-    total_ms = ev[0].elapsed_time(ev[K])
+    if graph is not None:
+        per = [ev[0].elapsed_time(ev[K]) / K] * K
+    elif scratch is not None:
+        per = [starts[i].elapsed_time(ev[i + 1]) for i in range(K)]
+    else:
+        per = [ev[i].elapsed_time(ev[i + 1]) for i in range(K)]
+    total_ms = sum(per) if scratch is not None else ev[0].elapsed_time(ev[K])
     t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -324,7 +347,9 @@ def run_ours(args):
             "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded normal draws, WAN2.2 shapes; no model weights)",
-            "config": dict(config_dict(w, spec, world), launch="cuda_graph" if graph is not None else "stream"),
+            "config": dict(config_dict(w, spec, world), launch="cuda_graph" if graph is not None else "stream",
+                           **({"l2": "flushed before every timed launch (512 MB write, outside the "
+                                     "per-launch events)"} if scratch is not None else {})),
             "rows_per_s": round(world * w.rows / (ms_step * 1e-3), 1),
             "pct_of_peak": round(100.0 * value / world / peak, 2),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
@@ -349,14 +374,14 @@ def run_e2e(args, w, spec, host, d, dev, world, local, fn, torch, dist):
     rows = w.rows
     chunk = 4096
     hy = torch.empty((w.B, w.L, w.D), dtype=torch.bfloat16, pin_memory=True)
-    hr = torch.empty_like(hy, pin_memory=True)
+    hr = None if spec.norm_only else torch.empty_like(hy, pin_memory=True)
     s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
     dy = torch.empty((w.B, w.L, w.D), dtype=torch.bfloat16, device=dev)
-    dr = torch.empty_like(dy)
+    dr = None if spec.norm_only else torch.empty_like(dy)
     per_row = {k: (w.layout(k) == "row") for k in ("gate", "scale", "shift")}
     flat = lambda t: t.view(-1, w.D)
     h2d_bytes = sum(v.numel() * 2 for v in host.values())
-    d2h_bytes = (hy.numel() + hr.numel()) * 2
+    d2h_bytes = (hy.numel() + (0 if hr is None else hr.numel())) * 2
 
     n_chunks = (rows + chunk - 1) // chunk
     kernel_done = [None] * n_chunks   # chunk c's kernel of the previous step
@@ -377,7 +402,8 @@ def run_e2e(args, w, spec, host, d, dev, world, local, fn, torch, dist):
                 if kernel_done[c] is not None:      # inputs of chunk c no longer read
                     s_in.wait_event(kernel_done[c])
                 for k in ("x", "residual") + tuple(k for k in ("gate", "scale", "shift") if per_row.get(k)):
-                    flat(d[k])[r0:r1].copy_(flat(host[k])[r0:r1], non_blocking=True)
+                    if k in host:
+                        flat(d[k])[r0:r1].copy_(flat(host[k])[r0:r1], non_blocking=True)
                 e_in = torch.cuda.Event()
                 e_in.record(s_in)
             s_cmp.wait_event(e_in)
@@ -385,19 +411,26 @@ def run_e2e(args, w, spec, host, d, dev, world, local, fn, torch, dist):
                 s_cmp.wait_event(copied_out[c])
             sub = lambda t, k: (flat(t)[r0:r1].view(1, r1 - r0, w.D) if per_row.get(k, True) else t)
             # a chunk of tokens is a (1, n, D) problem when B == 1 and there is no frame axis
-            fn.fused_residual_norm_scale_shift(
-                sub(d["residual"], "residual"), sub(d["x"], "x"),
-                sub(d["gate"], "gate") if "gate" in d else None, d.get("weight"), d.get("bias"),
-                sub(d["scale"], "scale"), sub(d["shift"], "shift"), norm, w.eps,
-                out=flat(dy)[r0:r1].view(1, r1 - r0, w.D),
-                residual_out=flat(dr)[r0:r1].view(1, r1 - r0, w.D), stream=s_cmp)
+            if spec.norm_only:
+                fn.norm_scale_shift(
+                    sub(d["x"], "x"), d.get("weight"), d.get("bias"), sub(d["scale"], "scale"),
+                    sub(d["shift"], "shift"), norm, w.eps,
+                    out=flat(dy)[r0:r1].view(1, r1 - r0, w.D), stream=s_cmp)
+            else:
+                fn.fused_residual_norm_scale_shift(
+                    sub(d["residual"], "residual"), sub(d["x"], "x"),
+                    sub(d["gate"], "gate") if "gate" in d else None, d.get("weight"), d.get("bias"),
+                    sub(d["scale"], "scale"), sub(d["shift"], "shift"), norm, w.eps,
+                    out=flat(dy)[r0:r1].view(1, r1 - r0, w.D),
+                    residual_out=flat(dr)[r0:r1].view(1, r1 - r0, w.D), stream=s_cmp)
             e_c = torch.cuda.Event()
             e_c.record(s_cmp)
             kernel_done[c] = e_c
             s_out.wait_event(e_c)
             with torch.cuda.stream(s_out):
                 flat(hy)[r0:r1].copy_(flat(dy)[r0:r1], non_blocking=True)
-                flat(hr)[r0:r1].copy_(flat(dr)[r0:r1], non_blocking=True)
+                if hr is not None:
+                    flat(hr)[r0:r1].copy_(flat(dr)[r0:r1], non_blocking=True)
                 e_o = torch.cuda.Event()
                 e_o.record(s_out)
             copied_out[c] = e_o
@@ -441,12 +474,14 @@ def _oracle_rows(w, spec, host_np, r0, r1):
     bst = lambda k: st if w.layout(k) == "row" else (0, 0, 0)
     sl = lambda k: host_np[k][r0:r1] if w.layout(k) == "row" else host_np[k]
     return oracle.fused_norm(1, n, w.D, x=host_np["x"][r0:r1], x_st=st,
-                             residual=host_np["residual"][r0:r1], res_st=st,
+                             residual=None if spec.norm_only else host_np["residual"][r0:r1],
+                             res_st=None if spec.norm_only else st,
                              gate=sl("gate") if spec.has_gate else None,
                              gate_st=bst("gate") if spec.has_gate else None,
                              weight=host_np.get("weight"), bias=host_np.get("bias"),
                              scale=sl("scale"), scale_st=bst("scale"), shift=sl("shift"),
-                             shift_st=bst("shift"), is_rms=spec.is_rms, eps=w.eps)
+                             shift_st=bst("shift"), is_rms=spec.is_rms, norm_only=spec.norm_only,
+                             eps=w.eps)
 
 
 def cpu_baseline(w, spec, host, seconds):
@@ -463,9 +498,33 @@ def cpu_baseline(w, spec, host, seconds):
         _oracle_rows(w, spec, host_np, done, r1)
         done = r1
     el = time.time() - t0
+    cores = oracle.num_threads()
+    # the same oracle on one core, over a 4096-row slice
+    n1 = min(4096, w.rows)
+    oracle.set_num_threads(1)
+    try:
+        t1 = time.time()
+        _oracle_rows(w, spec, host_np, 0, n1)
+        el1 = time.time() - t1
+    finally:
+        oracle.set_num_threads(cores)
     return {"value": round(done * per_row_bytes / el / 1e9, 4), "unit": "GB/s",
-            "rows_per_s": round(done / el, 1), "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"first {done} of {w.rows} rows of the same workload ({el:.1f} s)"}
+            "rows_per_s": round(done / el, 1), "cores": cores, "kind": "oracle",
+            "cpu_model": cpu_model(),
+            "sample": f"first {done} of {w.rows} rows of the same workload ({el:.1f} s)",
+            "one_core": {"value": round(n1 * per_row_bytes / el1 / 1e9, 4), "unit": "GB/s",
+                         "rows_per_s": round(n1 / el1, 1), "sample": f"first {n1} rows"}}
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
 
 
 def torch_int16():
@@ -489,7 +548,8 @@ def run_reference(args):
     # size the per-step sample so warm-up + timed steps take about 2 minutes
     budget_s = 120.0
     probe_rows = 512
-    names = ["x", "residual", "scale", "shift"] + (["gate"] if spec.has_gate else []) + \
+    names = ["x", "scale", "shift"] + ([] if spec.norm_only else ["residual"]) + \
+        (["gate"] if spec.has_gate and not spec.norm_only else []) + \
         (["weight"] if spec.has_weight else []) + (["bias"] if spec.has_bias else [])
 
     def gen(rows):

@@ -48,6 +48,8 @@ def _load():
     lib.oracle_fused_norm.restype = ctypes.c_int
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ctypes.c_int
+    lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+    lib.oracle_set_num_threads.restype = None
     _lib = lib
     return lib
 
@@ -63,6 +65,11 @@ def bf16_to_double(bits: int) -> float:
 
 def num_threads() -> int:
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads for the row loop of later calls (OpenMP)."""
+    _load().oracle_set_num_threads(int(n))
 
 
 def _p(a):

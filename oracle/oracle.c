@@ -176,6 +176,11 @@ int oracle_fused_norm(int64_t B, int64_t L, int64_t D, int64_t tokens_per_frame,
   return bad ? -1 : 0;
 }
 
+/* Threads the oracle's row loop uses from now on (n >= 1). Not part of the arithmetic. */
+void oracle_set_num_threads(int n) {
+  if (n >= 1) omp_set_num_threads(n);
+}
+
 int oracle_num_threads(void) {
   int n = 1;
 #pragma omp parallel

@@ -21,7 +21,8 @@ using namespace fused_norm_impl;
 
 struct fused_norm_s {
   fn_config cfg;
-  LaunchFn launch;
+  LaunchFn launch;            // scale or shift changes from token to token
+  LaunchFn launch_cached_mod;  // scale and shift both broadcast, per batch or per frame
   int threads;
 };
 
@@ -209,13 +210,13 @@ int64_t grid_for(int64_t rows) {
 
 namespace fused_norm_impl {
 LaunchFn select_launcher(int D, bool is_rms, bool norm_only, bool has_gate, bool has_weight,
-                         bool has_bias, bool f32) {
+                         bool has_bias, bool f32, bool cm) {
   if (D == 5120)
-    return is_rms ? select_launcher_5120_rms(norm_only, has_gate, has_weight, has_bias, f32)
-                  : select_launcher_5120_ln(norm_only, has_gate, has_weight, has_bias, f32);
+    return is_rms ? select_launcher_5120_rms(norm_only, has_gate, has_weight, has_bias, f32, cm)
+                  : select_launcher_5120_ln(norm_only, has_gate, has_weight, has_bias, f32, cm);
   if (D == 10240)
-    return is_rms ? select_launcher_10240_rms(norm_only, has_gate, has_weight, has_bias, f32)
-                  : select_launcher_10240_ln(norm_only, has_gate, has_weight, has_bias, f32);
+    return is_rms ? select_launcher_10240_rms(norm_only, has_gate, has_weight, has_bias, f32, cm)
+                  : select_launcher_10240_ln(norm_only, has_gate, has_weight, has_bias, f32, cm);
   return nullptr;
 }
 }  // namespace fused_norm_impl
@@ -233,12 +234,15 @@ fn_status fused_norm_create(fused_norm_t* out, const fn_config* cfg) {
   if (c.norm_only && c.has_gate) return FN_ERR_INVALID_ARG;
   if (c.D != 5120 && c.D != 10240) return FN_ERR_UNSUPPORTED;
   LaunchFn fn = select_launcher(c.D, c.is_rms, c.norm_only, c.has_gate, c.has_weight, c.has_bias,
-                                c.affine_fp32);
-  if (!fn) return FN_ERR_UNSUPPORTED;
+                                c.affine_fp32, false);
+  LaunchFn fn_cm = select_launcher(c.D, c.is_rms, c.norm_only, c.has_gate, c.has_weight, c.has_bias,
+                                   c.affine_fp32, true);
+  if (!fn || !fn_cm) return FN_ERR_UNSUPPORTED;
   fused_norm_s* h = new (std::nothrow) fused_norm_s;
   if (!h) return FN_ERR_INVALID_ARG;
   h->cfg = c;
   h->launch = fn;
+  h->launch_cached_mod = fn_cm;
   h->threads = c.D / (8 * (c.D == 5120 ? RowShape<5120>::VPT : RowShape<10240>::VPT));
   *out = h;
   return FN_OK;
@@ -261,7 +265,9 @@ fn_status fused_norm_launch(fused_norm_t h, const fn_args* a, fn_stream_t stream
   const int64_t rows = a->B * a->L;
   if (rows == 0) return FN_OK;
   RowParams p = make_params(h, a);
-  cudaError_t e = h->launch(p, grid_for(rows), reinterpret_cast<cudaStream_t>(stream));
+  const bool cached_mod = a->scale.stride_l == 0 && a->shift.stride_l == 0;
+  cudaError_t e = (cached_mod ? h->launch_cached_mod : h->launch)(p, grid_for(rows),
+                                                                  reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
     g_last_cuda_error = (int)e;
     return FN_ERR_CUDA;

@@ -26,6 +26,8 @@
 //     otherwise (a few in 10^4 elements) the element is recomputed in fp64 and
 //     rounded once (round-to-odd to fp32, then nearest-even to bf16). y is therefore
 //     the correctly rounded bf16 of the formula evaluated with the fp64 statistics.
+//     At D = 10240 the fp32 arithmetic runs two elements per instruction (sm_100
+//     f32x2), with results identical to the scalar form.
 //   * r is the correctly rounded bf16 of the exact residual + gate * x: gate * x is
 //     exact in fp32 (two 8-bit significands); when the fp32 sum lands exactly on a
 //     bf16 midpoint, TwoSum recovers the sum's rounding error and its sign decides.
@@ -202,6 +204,77 @@ __device__ __forceinline__ float y_fast_core(uint32_t vw, uint32_t sw, uint32_t 
   return y;
 }
 
+// ---- paired fp32 arithmetic (sm_100: two fp32 lanes per instruction, each lane
+// rounded as the scalar instruction would) ----------------------------------------
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ float bf16_mid(float y) {
+  return __uint_as_float((__float_as_uint(y) & 0xFFFF0000u) | 0x8000u);
+}
+
+// y_fast_core for both elements of one packed word (low half first): the same
+// operations in the same order, two lanes per instruction where no operand needs its
+// magnitude, so each y, bound and decision is bit-identical to the scalar path.
+template <bool HAS_WEIGHT, bool HAS_BIAS>
+__device__ __forceinline__ void y_fast_pair(uint32_t vw, uint32_t sw, uint32_t tw, float w0, float w1,
+                                            float b0, float b1, const RowStats& st, float& y0,
+                                            float& y1, bool& near0, bool& near1) {
+  constexpr float k8u = 4.76837158203125e-7f;  // 2^-21
+  constexpr float kEdge = 9.765625e-4f;        // 2^-10
+  const uint64_t n = mul2(pk2(add_bf16_f32<0>(vw, st.neg_mu32), add_bf16_f32<1>(vw, st.neg_mu32)),
+                          pk2(st.rho32, st.rho32));
+  const uint64_t nw = HAS_WEIGHT ? mul2(n, pk2(w0, w1)) : n;
+  const uint64_t nb = HAS_BIAS ? add2(nw, pk2(b0, b1)) : nw;
+  const float a0 = add_bf16_f32<0>(sw, 1.0f), a1 = add_bf16_f32<1>(sw, 1.0f);
+  const float t0 = lo_f(tw), t1 = hi_f(tw);
+  const uint64_t y = fma2(nb, pk2(a0, a1), pk2(t0, t1));
+  float nw0, nw1;
+  upk2(nw, nw0, nw1);
+  float in0 = HAS_WEIGHT ? fmaf(fabsf(w0), st.kappa, fabsf(nw0)) : st.kappa + fabsf(nw0);
+  float in1 = HAS_WEIGHT ? fmaf(fabsf(w1), st.kappa, fabsf(nw1)) : st.kappa + fabsf(nw1);
+  if (HAS_BIAS) {
+    in0 += fabsf(b0);
+    in1 += fabsf(b1);
+  }
+  const uint64_t bound = mul2(pk2(fmaf(fabsf(a0), in0, fabsf(t0)), fmaf(fabsf(a1), in1, fabsf(t1))),
+                              pk2(k8u, k8u));
+  upk2(y, y0, y1);
+  const uint64_t dm = sub2(y, pk2(bf16_mid(y0), bf16_mid(y1)));
+  const uint64_t ye = mul2(y, pk2(kEdge, kEdge));
+  float d0, d1, e0, e1, q0, q1;
+  upk2(dm, d0, d1);
+  upk2(ye, e0, e1);
+  upk2(bound, q0, q1);
+  near0 |= !(fminf(fabsf(d0), fabsf(e0)) > q0);
+  near1 |= !(fminf(fabsf(d1), fabsf(e1)) > q1);
+}
+
 // y_fast_core with bf16 weight / bias taken from packed words.
 template <int H, bool HAS_WEIGHT, bool HAS_BIAS>
 __device__ __forceinline__ float y_fast(uint32_t vw, uint32_t sw, uint32_t tw, uint32_t ww,
@@ -218,7 +291,7 @@ __device__ __forceinline__ float elem_dyn(const uint4& v, int q) {
 
 // One 16-byte vector of y: the fp32 fast path for all eight elements, then (rarely) the
 // fp64 path for the elements whose fast value came near a rounding boundary.
-template <bool HAS_WEIGHT, bool HAS_BIAS>
+template <bool PAIRED, bool HAS_WEIGHT, bool HAS_BIAS>
 __device__ __forceinline__ uint4 output_vec(const uint4& v, const uint4& sv, const uint4& tv,
                                             const uint4& wv, const uint4& bv, const RowStats& st) {
   uint32_t o[4];
@@ -228,8 +301,14 @@ __device__ __forceinline__ uint4 output_vec(const uint4& v, const uint4& sv, con
     const uint32_t vw = word(v, i), sw = word(sv, i), tw = word(tv, i);
     const uint32_t ww = word(wv, i), bw = word(bv, i);
     bool n0 = false, n1 = false;
-    const float y0 = y_fast<0, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, ww, bw, st, n0);
-    const float y1 = y_fast<1, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, ww, bw, st, n1);
+    float y0, y1;
+    if (PAIRED) {
+      y_fast_pair<HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, lo_f(ww), hi_f(ww), lo_f(bw), hi_f(bw), st, y0, y1,
+                                        n0, n1);
+    } else {
+      y0 = y_fast<0, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, ww, bw, st, n0);
+      y1 = y_fast<1, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, ww, bw, st, n1);
+    }
     o[i] = pack_rn(y0, y1);
     near_mask |= (n0 ? 1u : 0u) << (2 * i);
     near_mask |= (n1 ? 2u : 0u) << (2 * i);
@@ -268,7 +347,7 @@ __device__ __forceinline__ float sel8(const Affine8& a, int q) {
 }
 
 // As output_vec, with fp32 weight / bias.
-template <bool HAS_WEIGHT, bool HAS_BIAS>
+template <bool PAIRED, bool HAS_WEIGHT, bool HAS_BIAS>
 __device__ __forceinline__ uint4 output_vec_f32(const uint4& v, const uint4& sv, const uint4& tv,
                                                 const Affine8& wf, const Affine8& bf,
                                                 const RowStats& st) {
@@ -278,8 +357,14 @@ __device__ __forceinline__ uint4 output_vec_f32(const uint4& v, const uint4& sv,
   for (int i = 0; i < 4; ++i) {
     const uint32_t vw = word(v, i), sw = word(sv, i), tw = word(tv, i);
     bool n0 = false, n1 = false;
-    const float y0 = y_fast_core<0, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, wf.v[2 * i], bf.v[2 * i], st, n0);
-    const float y1 = y_fast_core<1, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, wf.v[2 * i + 1], bf.v[2 * i + 1], st, n1);
+    float y0, y1;
+    if (PAIRED) {
+      y_fast_pair<HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, wf.v[2 * i], wf.v[2 * i + 1], bf.v[2 * i],
+                                        bf.v[2 * i + 1], st, y0, y1, n0, n1);
+    } else {
+      y0 = y_fast_core<0, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, wf.v[2 * i], bf.v[2 * i], st, n0);
+      y1 = y_fast_core<1, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, wf.v[2 * i + 1], bf.v[2 * i + 1], st, n1);
+    }
     o[i] = pack_rn(y0, y1);
     near_mask |= (n0 ? 1u : 0u) << (2 * i);
     near_mask |= (n1 ? 2u : 0u) << (2 * i);
@@ -318,18 +403,48 @@ template <int D> struct RowShape;
 #ifndef FN_MINB_10240
 #define FN_MINB_10240 2
 #endif
+// 1: y's fp32 arithmetic in paired (f32x2) instructions. Bit-identical either way; it
+// cuts ~6% of the instructions but lengthens each thread's dependency chains. Measured
+// on B200: ~4% faster at D = 10240 (two CTAs per SM, issue-bound with weight), neutral
+// to mixed at D = 5120 and slower there when launches run serialised.
+// CTAs per SM for the instances whose scale and shift are broadcast or per frame: they
+// fetch scale and shift from L1 as each vector is used instead of holding them across
+// the statistics, which frees registers for more rows per SM (measured on B200: frame
+// gate, broadcast fused and norm-only shapes 2-5% faster than with the streamed
+// instances; 7 CTAs at D = 5120 is slower again).
+#ifndef FN_MINB_CM_5120
+#define FN_MINB_CM_5120 6
+#endif
+#ifndef FN_MINB_CM_10240
+#define FN_MINB_CM_10240 3
+#endif
+#ifndef FN_PAIRED_5120
+#define FN_PAIRED_5120 0
+#endif
+#ifndef FN_PAIRED_10240
+#define FN_PAIRED_10240 1
+#endif
 // 1: scale/shift loads are issued with x and residual, before the r stores;
 // 0: after them, where the statistics' reduction and barrier hide their latency
 // (fewer live registers; measured faster on B200 for the WAN2.2 shape).
 #ifndef FN_EARLY_MODULATION_LOADS
 #define FN_EARLY_MODULATION_LOADS 0
 #endif
-template <> struct RowShape<5120> { static constexpr int VPT = FN_VPT_5120, kMinBlocks = FN_MINB_5120; };
-template <> struct RowShape<10240> { static constexpr int VPT = FN_VPT_10240, kMinBlocks = FN_MINB_10240; };
+template <> struct RowShape<5120> {
+  static constexpr int VPT = FN_VPT_5120, kMinBlocks = FN_MINB_5120;
+  static constexpr int kMinBlocksCachedMod = FN_MINB_CM_5120;
+  static constexpr bool kPaired = FN_PAIRED_5120 != 0;
+};
+template <> struct RowShape<10240> {
+  static constexpr int VPT = FN_VPT_10240, kMinBlocks = FN_MINB_10240;
+  static constexpr int kMinBlocksCachedMod = FN_MINB_CM_10240;
+  static constexpr bool kPaired = FN_PAIRED_10240 != 0;
+};
 
 template <int D, int VPT, bool IS_RMS, bool NORM_ONLY, bool HAS_GATE, bool HAS_WEIGHT, bool HAS_BIAS,
-          bool AFFINE_F32>
-__global__ void __launch_bounds__(D / (8 * VPT), RowShape<D>::kMinBlocks)
+          bool AFFINE_F32, bool CACHED_MOD>
+__global__ void __launch_bounds__(D / (8 * VPT), CACHED_MOD ? RowShape<D>::kMinBlocksCachedMod
+                                                            : RowShape<D>::kMinBlocks)
 fused_norm_rows(const RowParams p) {
   constexpr int T = D / (8 * VPT);
   constexpr int W = T / 32;
@@ -368,7 +483,7 @@ fused_norm_rows(const RowParams p) {
 #pragma unroll
       for (int k = 0; k < VPT; ++k) gv[k] = load_vec(gr, tid + k * T, p.stream_mask & kGate);
     }
-    if (FN_EARLY_MODULATION_LOADS) {
+    if (FN_EARLY_MODULATION_LOADS && !CACHED_MOD) {
 #pragma unroll
       for (int k = 0; k < VPT; ++k) {
         sv[k] = load_vec(sr, tid + k * T, p.stream_mask & kScale);
@@ -390,7 +505,7 @@ fused_norm_rows(const RowParams p) {
       }
     }
 
-    if (!FN_EARLY_MODULATION_LOADS) {
+    if (!FN_EARLY_MODULATION_LOADS && !CACHED_MOD) {
 #pragma unroll
       for (int k = 0; k < VPT; ++k) {
         sv[k] = load_vec(sr, tid + k * T, p.stream_mask & kScale);
@@ -476,67 +591,78 @@ fused_norm_rows(const RowParams p) {
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
       const int j = tid + k * T;
+      if (CACHED_MOD) {  // broadcast / per-frame rows: L1 hits, fetched as they are used
+        sv[k] = __ldg(reinterpret_cast<const uint4*>(sr) + j);
+        tv[k] = __ldg(reinterpret_cast<const uint4*>(tr) + j);
+      }
       if (AFFINE_F32) {
         Affine8 wf{{1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f}}, bf{{0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}};
         if (HAS_WEIGHT) wf = load_affine_f32(p.weight, j);
         if (HAS_BIAS) bf = load_affine_f32(p.bias, j);
-        __stcs(yo + j, output_vec_f32<HAS_WEIGHT, HAS_BIAS>(v[k], sv[k], tv[k], wf, bf, st));
+        __stcs(yo + j, output_vec_f32<RowShape<D>::kPaired, HAS_WEIGHT, HAS_BIAS>(v[k], sv[k], tv[k], wf, bf, st));
       } else {
         uint4 wv = make_uint4(0, 0, 0, 0), bv = make_uint4(0, 0, 0, 0);
         if (HAS_WEIGHT) wv = __ldg(reinterpret_cast<const uint4*>(p.weight) + j);
         if (HAS_BIAS) bv = __ldg(reinterpret_cast<const uint4*>(p.bias) + j);
-        __stcs(yo + j, output_vec<HAS_WEIGHT, HAS_BIAS>(v[k], sv[k], tv[k], wv, bv, st));
+        __stcs(yo + j, output_vec<RowShape<D>::kPaired, HAS_WEIGHT, HAS_BIAS>(v[k], sv[k], tv[k], wv, bv, st));
       }
     }
   }
 }
 
 template <int D, int VPT, bool IS_RMS, bool NORM_ONLY, bool HAS_GATE, bool HAS_WEIGHT, bool HAS_BIAS,
-          bool AFFINE_F32>
+          bool AFFINE_F32, bool CACHED_MOD>
 cudaError_t launch_rows(const RowParams& p, int64_t grid, cudaStream_t stream) {
   constexpr int T = D / (8 * VPT);
-  fused_norm_rows<D, VPT, IS_RMS, NORM_ONLY, HAS_GATE, HAS_WEIGHT, HAS_BIAS, AFFINE_F32>
+  fused_norm_rows<D, VPT, IS_RMS, NORM_ONLY, HAS_GATE, HAS_WEIGHT, HAS_BIAS, AFFINE_F32, CACHED_MOD>
       <<<(unsigned)grid, T, 0, stream>>>(p);
   return cudaGetLastError();
 }
 
-// Launcher for one (norm_only, gate) group: the affine combinations.
-template <int D, bool RMS, bool NO, bool G>
+// Launcher for one (norm_only, gate, modulation caching) group: the affine combinations.
+template <int D, bool RMS, bool NO, bool G, bool CM>
 LaunchFn pick_affine(bool w, bool b, bool f32) {
   constexpr int V = RowShape<D>::VPT;
-  if (!w && !b) return &launch_rows<D, V, RMS, NO, G, false, false, false>;
+  if (!w && !b) return &launch_rows<D, V, RMS, NO, G, false, false, false, CM>;
   if (f32) {
-    if (w && b) return &launch_rows<D, V, RMS, NO, G, true, true, true>;
-    return w ? &launch_rows<D, V, RMS, NO, G, true, false, true>
-             : &launch_rows<D, V, RMS, NO, G, false, true, true>;
+    if (w && b) return &launch_rows<D, V, RMS, NO, G, true, true, true, CM>;
+    return w ? &launch_rows<D, V, RMS, NO, G, true, false, true, CM>
+             : &launch_rows<D, V, RMS, NO, G, false, true, true, CM>;
   }
-  if (w && b) return &launch_rows<D, V, RMS, NO, G, true, true, false>;
-  return w ? &launch_rows<D, V, RMS, NO, G, true, false, false>
-           : &launch_rows<D, V, RMS, NO, G, false, true, false>;
+  if (w && b) return &launch_rows<D, V, RMS, NO, G, true, true, false, CM>;
+  return w ? &launch_rows<D, V, RMS, NO, G, true, false, false, CM>
+           : &launch_rows<D, V, RMS, NO, G, false, true, false, CM>;
 }
 
 // Launcher for every specialisation of one (D, norm); instantiated in one translation
-// unit per (D, norm) so the instances compile in parallel.
+// unit per (D, norm) so the instances compile in parallel. cached_mod selects the
+// instances for scale and shift that are broadcast or per frame (re-read by many rows).
 template <int D, bool RMS>
-LaunchFn pick_launcher(bool norm_only, bool has_gate, bool has_weight, bool has_bias, bool f32) {
-  if (norm_only) return pick_affine<D, RMS, true, false>(has_weight, has_bias, f32);
-  return has_gate ? pick_affine<D, RMS, false, true>(has_weight, has_bias, f32)
-                  : pick_affine<D, RMS, false, false>(has_weight, has_bias, f32);
+LaunchFn pick_launcher(bool norm_only, bool has_gate, bool has_weight, bool has_bias, bool f32,
+                       bool cached_mod) {
+  if (cached_mod) {
+    if (norm_only) return pick_affine<D, RMS, true, false, true>(has_weight, has_bias, f32);
+    return has_gate ? pick_affine<D, RMS, false, true, true>(has_weight, has_bias, f32)
+                    : pick_affine<D, RMS, false, false, true>(has_weight, has_bias, f32);
+  }
+  if (norm_only) return pick_affine<D, RMS, true, false, false>(has_weight, has_bias, f32);
+  return has_gate ? pick_affine<D, RMS, false, true, false>(has_weight, has_bias, f32)
+                  : pick_affine<D, RMS, false, false, false>(has_weight, has_bias, f32);
 }
 
 LaunchFn select_launcher(int D, bool is_rms, bool norm_only, bool has_gate, bool has_weight,
-                         bool has_bias, bool affine_f32);
-LaunchFn select_launcher_5120_ln(bool norm_only, bool has_gate, bool has_weight, bool has_bias, bool f32);
-LaunchFn select_launcher_5120_rms(bool norm_only, bool has_gate, bool has_weight, bool has_bias, bool f32);
-LaunchFn select_launcher_10240_ln(bool norm_only, bool has_gate, bool has_weight, bool has_bias, bool f32);
-LaunchFn select_launcher_10240_rms(bool norm_only, bool has_gate, bool has_weight, bool has_bias, bool f32);
+                         bool has_bias, bool affine_f32, bool cached_mod);
+LaunchFn select_launcher_5120_ln(bool norm_only, bool has_gate, bool has_weight, bool has_bias, bool f32, bool cm);
+LaunchFn select_launcher_5120_rms(bool norm_only, bool has_gate, bool has_weight, bool has_bias, bool f32, bool cm);
+LaunchFn select_launcher_10240_ln(bool norm_only, bool has_gate, bool has_weight, bool has_bias, bool f32, bool cm);
+LaunchFn select_launcher_10240_rms(bool norm_only, bool has_gate, bool has_weight, bool has_bias, bool f32, bool cm);
 
 }  // namespace fused_norm_impl
 
 // Defines the launcher selector of one (D, norm) translation unit.
 #define FUSED_NORM_DEFINE_SELECTOR(NAME, D_, RMS_)                                              \
   namespace fused_norm_impl {                                                                   \
-  LaunchFn NAME(bool norm_only, bool has_gate, bool has_weight, bool has_bias, bool f32) {      \
-    return pick_launcher<D_, RMS_>(norm_only, has_gate, has_weight, has_bias, f32);             \
+  LaunchFn NAME(bool norm_only, bool has_gate, bool has_weight, bool has_bias, bool f32, bool cm) { \
+    return pick_launcher<D_, RMS_>(norm_only, has_gate, has_weight, has_bias, f32, cm);         \
   }                                                                                             \
   }

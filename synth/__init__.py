@@ -311,6 +311,13 @@ W5B = _add(Workload("frame_gate_B1_F49x3600_D5120", 1, 176400, 5120, 49,
 W6 = _add(Workload("batch_bcast_B3_L64_D5120", 3, 64, 5120, 0,
                    (("gate", "batch"), ("scale", "batch"), ("shift", "batch")), _DISTS,
                    (Spec(False, True, True), Spec(True, True, False)), seed=1007))
+# The pages' own microbenchmark shape (sglang PR #36349, "Microbenchmark"): LayerNorm,
+# seq 176400, dim 5120, gate, scale and shift broadcast (1, 1, D); the fused op without
+# and with an affine weight and bias, and the norm-only op.
+W7 = _add(Workload("microbench_bcast_B1_L176400_D5120", 1, 176400, 5120, 0,
+                   (("gate", "bcast"), ("scale", "bcast"), ("shift", "bcast")), _DISTS,
+                   (Spec(False, True, False), Spec(False, True, True, has_bias=True),
+                    Spec(False, False, False, norm_only=True)), seed=1008))
 
 
 def scaled(w: Workload, L: int, name: Optional[str] = None, F: Optional[int] = None) -> Workload:

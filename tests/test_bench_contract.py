@@ -49,3 +49,22 @@ def test_gpu_arm_line():
     assert e["value"] > 0 and e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["config"]["launch"] == "stream"
+    cb = d["cpu_baseline"]
+    assert cb["one_core"]["value"] > 0 and cb["one_core"]["rows_per_s"] > 0
+
+
+@pytest.mark.gpu
+def test_gpu_arm_flushed_small_case():
+    # a launch-bound shape with L2 flushed before every timed launch
+    d = _run(["--workload", "rms_fused_B1_L16_D5120", "--flush-l2", "--steps", "20", "--warmup", "5",
+              "--no-e2e", "--no-cpu-baseline"])
+    assert d["gpu_launches"] == 20 and d["value"] > 0
+    assert d["config"]["l2"].startswith("flushed")
+
+
+@pytest.mark.gpu
+def test_gpu_arm_norm_only():
+    d = _run(["--workload", "microbench_bcast_B1_L176400_D5120", "--spec", "ln_nss_now",
+              "--rows", "4096", "--steps", "10", "--warmup", "3", "--cpu-seconds", "1"])
+    assert d["config"]["spec"] == "ln_nss_now" and d["value"] > 0
+    assert d["e2e"]["d2h_bytes_per_step"] == 4096 * 5120 * 2   # y only

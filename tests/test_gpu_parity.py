@@ -75,6 +75,24 @@ def test_extra_layouts(w):
         _assert(*check_workload(w, spec, DEV), f"{w.name}/{spec.name}")
 
 
+@pytest.mark.parametrize("D", [5120, 10240])
+@pytest.mark.parametrize("layouts", [("bcast", "bcast", "bcast"), ("batch", "batch", "bcast"),
+                                     ("row", "bcast", "row"), ("bcast", "row", "bcast")],
+                         ids=lambda l: "-".join(l))
+def test_modulation_layouts(D, layouts):
+    # scale and shift broadcast or per batch run the instances that fetch them from L1 as
+    # they are used; one of them per token runs the instances that load them with x
+    base = synth.W3 if D == 5120 else synth.W3B
+    w = synth.scaled(base, 531)
+    w = synth.dataclasses.replace(w, B=2, layouts=(("gate", layouts[0]), ("scale", layouts[1]),
+                                                   ("shift", layouts[2])),
+                                  name=f"{w.name}_B2_{'-'.join(layouts)}")
+    for spec in (synth.Spec(False, True, False), synth.Spec(True, True, True),
+                 synth.Spec(False, False, True, has_bias=True),
+                 synth.Spec(True, False, True, norm_only=True)):
+        _assert(*check_workload(w, spec, DEV), f"{w.name}/{spec.name}")
+
+
 # ---- full-size configs --------------------------------------------------------
 
 @pytest.mark.parametrize("D", [5120, 10240])
@@ -109,6 +127,17 @@ def test_frame_gate_B1_F21x8400_full():
 
 def test_frame_gate_B1_F49x3600_full():
     _full_size(synth.W5B)
+
+
+@pytest.mark.parametrize("spec", synth.W7.specs, ids=lambda s: s.name)
+def test_microbench_bcast_B1_L176400_full(spec):
+    w = synth.W7
+    host = host_inputs(w, ("x", "residual", "gate", "scale", "shift", "weight", "bias"))
+    dev = upload_host(w, host, DEV)
+    ty, tr = check_workload(w, spec, DEV, dev=dev, host=host)
+    del dev, host
+    torch.cuda.empty_cache()
+    _assert(ty, tr, f"{w.name}/{spec.name}")
 
 
 # ---- fp32 affine parameters ----------------------------------------------------------
