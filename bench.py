@@ -100,13 +100,40 @@ def config_dict(w, spec, n):
                   else "L2-resident (small case)"}
 
 
+def _code_tokens(src: str) -> str:
+    """C/C++ source with comments removed and whitespace runs collapsed (string and
+    character literals kept verbatim): what the compiler sees, not how it is annotated."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        elif c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_digest():
+    """sha256 over the kernel sources' code (comments and layout excluded), so that a
+    recorded ncu measurement stays attached to the code it was taken on."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "rmsnorm_row_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".cuh", ".h")):
             h.update(name.encode())
-            h.update(open(os.path.join(csrc, name), "rb").read())
+            h.update(_code_tokens(open(os.path.join(csrc, name), encoding="utf-8").read()).encode())
     return h.hexdigest()
 
 

@@ -28,12 +28,13 @@
 //     the correctly rounded bf16 of the formula evaluated with the fp64 statistics.
 //     At D = 10240 the fp32 arithmetic runs two elements per instruction (sm_100
 //     f32x2), with results identical to the scalar form.
-//   * r is the correctly rounded bf16 of the exact residual + gate * x: gate * x is
-//     exact in fp32 (two 8-bit significands); when the fp32 sum lands exactly on a
-//     bf16 midpoint, TwoSum recovers the sum's rounding error and its sign decides.
+//   * r is the correctly rounded bf16 of the exact residual + gate * x: one bf16x2
+//     fused multiply-add per pair computes the exact value and rounds it once.
 //   * Per-row (streamed-once) operands use evict-first loads and stores; broadcast
 //     and per-frame operands use the read-only cached path (they are re-read by
-//     every row and stay in L1/L2).
+//     every row and stay in L1/L2). When scale and shift are both of the second kind,
+//     separate instances fetch them as each vector is used rather than holding them
+//     across the statistics, and run one more CTA per SM on the registers saved.
 #pragma once
 
 #include <cuda_bf16.h>

@@ -68,3 +68,16 @@ def test_gpu_arm_norm_only():
               "--rows", "4096", "--steps", "10", "--warmup", "3", "--cpu-seconds", "1"])
     assert d["config"]["spec"] == "ln_nss_now" and d["value"] > 0
     assert d["e2e"]["d2h_bytes_per_step"] == 4096 * 5120 * 2   # y only
+
+
+def test_kernel_digest_ignores_comments_only():
+    # the recorded ncu traffic stays attached to the code it was measured on: comments
+    # and layout do not change the digest, code does (string literals kept verbatim)
+    sys.path.insert(0, ROOT)
+    import bench
+    base = 'x = a + b; // sum\nasm("add.f32 %0, %1; // not a comment");'
+    assert bench._code_tokens(base) == bench._code_tokens(
+        '/* block */ x = a +   b;\n\nasm("add.f32 %0, %1; // not a comment"); // more')
+    assert bench._code_tokens(base) != bench._code_tokens(base.replace("a + b", "a - b"))
+    assert bench._code_tokens(base) != bench._code_tokens(base.replace("// not a", "// NOT a"))
+    assert bench._code_tokens("c = '\\''; // q") == "c = '\\'';"
