@@ -25,7 +25,6 @@ import argparse
 import datetime
 import hashlib
 import json
-import math
 import os
 import re
 import statistics

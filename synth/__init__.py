@@ -24,7 +24,7 @@ import ctypes
 import dataclasses
 import math
 import os
-from typing import Dict, Optional, Sequence, Tuple
+from typing import Dict, Optional, Tuple
 
 import numpy as np
 

@@ -13,7 +13,7 @@ import torch
 
 import rmsnorm_row_b200 as fn
 import synth
-from parity import Tally, check_workload, host_inputs, run_gpu, upload_host
+from parity import Tally, check_workload, host_inputs, upload_host
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda:0")
