@@ -77,15 +77,18 @@ def test_extra_layouts(w):
 
 @pytest.mark.parametrize("D", [5120, 10240])
 @pytest.mark.parametrize("layouts", [("bcast", "bcast", "bcast"), ("batch", "batch", "bcast"),
+                                     ("frame", "frame", "frame"), ("row", "frame", "bcast"),
                                      ("row", "bcast", "row"), ("bcast", "row", "bcast")],
                          ids=lambda l: "-".join(l))
 def test_modulation_layouts(D, layouts):
-    # scale and shift broadcast or per batch run the instances that fetch them from L1 as
-    # they are used; one of them per token runs the instances that load them with x
+    # scale and shift broadcast, per batch or per frame run the instances that fetch them
+    # from L1 as they are used; one of them per token runs the instances that load them
+    # with x. L = 531 = 9 frames of 59 tokens.
     base = synth.W3 if D == 5120 else synth.W3B
     w = synth.scaled(base, 531)
-    w = synth.dataclasses.replace(w, B=2, layouts=(("gate", layouts[0]), ("scale", layouts[1]),
-                                                   ("shift", layouts[2])),
+    w = synth.dataclasses.replace(w, B=2, F=9 if "frame" in layouts else 0,
+                                  layouts=(("gate", layouts[0]), ("scale", layouts[1]),
+                                           ("shift", layouts[2])),
                                   name=f"{w.name}_B2_{'-'.join(layouts)}")
     for spec in (synth.Spec(False, True, False), synth.Spec(True, True, True),
                  synth.Spec(False, False, True, has_bias=True),
