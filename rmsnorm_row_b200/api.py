@@ -15,6 +15,10 @@ fallback path).
 weight and bias are (D,) vectors, bf16 or fp32 (both the same dtype when both are given);
 fp32 values are used at full precision.
 
+Calls are asynchronous on `stream` (default: the current stream of the inputs' device),
+like any PyTorch kernel: when `stream` is not the stream the tensors were produced on, the
+caller orders the two streams and keeps the tensors alive (e.g. Tensor.record_stream).
+
 Accepted operand shapes for gate / scale / shift against x of shape (B, L, D):
     (D,), (1, D), (1, 1, D)      broadcast
     (B, L, D)                    per token
