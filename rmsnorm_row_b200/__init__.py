@@ -8,8 +8,9 @@ this package is a thin binding over it:
   the ctypes structures ``fn_config`` / ``fn_operand`` / ``fn_args``;
 * tensor-level ops ``fused_residual_norm_scale_shift`` and ``norm_scale_shift``.
 
-Importing needs the built library (``python -m rmsnorm_row_b200.build``); there is
-no fallback implementation.
+The library is loaded on first use: every entry point raises ImportError if it has not
+been built (``python -m rmsnorm_row_b200.build``); there is no fallback implementation.
+Importing the package does not need it, so the build module can run from a clean tree.
 """
 from ._abi import (FN_ERR_CUDA, FN_ERR_INVALID_ARG, FN_ERR_MISALIGNED, FN_ERR_UNSUPPORTED, FN_OK,
                    FusedNormError, fn_args, fn_config, fn_operand, fused_norm_create,
@@ -17,8 +18,6 @@ from ._abi import (FN_ERR_CUDA, FN_ERR_INVALID_ARG, FN_ERR_MISALIGNED, FN_ERR_UN
                    fused_norm_launch, fused_norm_plan, fused_norm_status_string,
                    fused_norm_validate, fused_norm_version, load)
 from .api import build_args, fused_residual_norm_scale_shift, norm_scale_shift
-
-load()
 
 __all__ = [
     "FN_OK", "FN_ERR_INVALID_ARG", "FN_ERR_UNSUPPORTED", "FN_ERR_MISALIGNED", "FN_ERR_CUDA",

@@ -249,3 +249,14 @@ def test_fp32_affine_extent_in_overlap_rules():
     a.y_stride_b, a.y_stride_l = 8 * 5120, 5120
     assert fn.fused_norm_validate(h16, a) == OK
     assert fn.fused_norm_validate(h32, a) == INV
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    # no fallback: without the built library every entry point raises, naming the build step
+    from rmsnorm_row_b200 import _abi
+    monkeypatch.setattr(_abi, "_lib", None)
+    monkeypatch.setattr(_abi, "LIB_PATH", str(tmp_path / "libfused_norm.so"))
+    with pytest.raises(ImportError, match="rmsnorm_row_b200.build"):
+        _abi.fused_norm_version()
+    with pytest.raises(ImportError, match="no fallback"):
+        _abi.fused_norm_create(_abi.fn_config(D=5120, eps=1e-6))
