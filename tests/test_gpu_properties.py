@@ -55,6 +55,28 @@ def test_hand_cases_exact(case, D):
 # ---- closed forms and identities ------------------------------------------------------
 
 @pytest.mark.parametrize("D", [5120, 10240])
+@pytest.mark.parametrize("op", ["norm_only", "fused"])
+def test_y_is_rounded_once(D, op):
+    # RMSNorm, eps = 0, rows of +-1: n = +-1 exactly and y = n (1 + 2^-8) + 2^-40. The
+    # positive elements lie just above the bf16 midpoint 1 + 2^-8 by less than float32
+    # resolution and must round up to 1 + 2^-7 (0x3F81), not to the float32 tie and then
+    # to the even 1.0; the negative ones round to -1.0 (0xBF80).
+    L = 4
+    row = torch.tensor([1.0, -1.0] * (D // 2))
+    v = row.repeat(1, L, 1).to(torch.bfloat16).to(DEV)
+    scale = torch.full((1, 1, D), 2.0 ** -8).to(torch.bfloat16).to(DEV)
+    shift = torch.full((1, 1, D), 2.0 ** -40).to(torch.bfloat16).to(DEV)
+    if op == "norm_only":
+        y = fn.norm_scale_shift(v, None, None, scale, shift, "rms", 0.0)
+    else:
+        y, _ = fn.fused_residual_norm_scale_shift(v, torch.zeros_like(v), None, None, None, scale,
+                                                  shift, "rms", 0.0)
+    torch.cuda.synchronize()
+    want = np.where(row.numpy() > 0, 0x3F81, 0xBF80).astype(np.uint16)
+    assert np.array_equal(bits(y)[0], np.tile(want, (L, 1)))
+
+
+@pytest.mark.parametrize("D", [5120, 10240])
 def test_constant_rows_give_shift_exactly(D):
     L = 64
     vals = torch.tensor([0.0, 1.0, -3.5, 0.15625, 96.0, 1e-3, -250.0, 7.0] * 8)[:L]

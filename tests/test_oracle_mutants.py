@@ -35,6 +35,17 @@ MUTANTS = [
     ("ties_away", "(frac == 0.5 && fmod(whole, 2.0) == 1.0)", "(frac == 0.5)", 0),
     ("rounding_truncates", "if (frac > 0.5 || (frac == 0.5 && fmod(whole, 2.0) == 1.0)) whole += 1.0;", "", 0),
     ("subnormal_quantum", "if (qexp < -133) qexp = -133;", "if (qexp < -126) qexp = -126;", 0),
+    ("bias_before_weight",
+     "        if (weight) n = n * oracle_bf16_to_double(weight[c]);\n"
+     "        if (weight_f32) n = n * (double)weight_f32[c];\n"
+     "        if (bias) n = n + oracle_bf16_to_double(bias[c]);\n",
+     "        if (bias) n = n + oracle_bf16_to_double(bias[c]);\n"
+     "        if (weight) n = n * oracle_bf16_to_double(weight[c]);\n"
+     "        if (weight_f32) n = n * (double)weight_f32[c];\n", 0),
+    ("norm_of_x_not_r", "v[c] = oracle_bf16_to_double(rb);", "v[c] = oracle_bf16_to_double(xr[c]);", 0),
+    ("rms_with_layernorm_statistics", "if (is_rms) {", "if (0) {", 0),
+    ("double_rounding_y", "yr[c] = oracle_bf16_rne(yv);", "yr[c] = oracle_bf16_rne((double)(float)yv);", 0),
+    ("batch_stride_ignored", "return b * st[0] + f * st[1] + l * st[2];", "return f * st[1] + l * st[2];", 0),
 ]
 
 

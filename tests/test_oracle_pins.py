@@ -281,6 +281,22 @@ def test_residual_rounding_near_tie_from_a_tiny_residual():
         assert np.all(bf16_bits_to_f64(out["r"][0, 0]) == want)
 
 
+def test_y_is_rounded_once():
+    # RMSNorm with eps = 0 of a row of +-1 gives n = +-1 exactly, so y = n (1 + s) + t is
+    # known exactly. With s = 2^-8 and t = 2^-40, y = 1 + 2^-8 + 2^-40 lies just above the
+    # bf16 midpoint 1 + 2^-8 (between 1 and 1 + 2^-7), by far less than float32
+    # resolution: one rounding gives 1 + 2^-7 (0x3F81); rounding through float32 first
+    # lands on the tie and then on the even neighbour 1.0 (0x3F80). The negative
+    # elements sit just inside the midpoint and round to -1.0 either way.
+    D = 8
+    r = np.array([1.0, -1.0] * (D // 2))
+    out = one_row(r, scale=np.full(D, 2.0 ** -8), shift=np.full(D, 2.0 ** -40), is_rms=True,
+                  eps=0.0)
+    assert np.array_equal(out["n"].reshape(D), r)
+    y = out["y"].reshape(D)
+    assert np.array_equal(y, np.where(r > 0, 0x3F81, 0xBF80).astype(np.uint16))
+
+
 def test_norm_only_equals_fused_with_zero_x():
     D = 80
     rng = np.random.default_rng(6)
