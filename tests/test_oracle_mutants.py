@@ -46,6 +46,10 @@ MUTANTS = [
     ("rms_with_layernorm_statistics", "if (is_rms) {", "if (0) {", 0),
     ("double_rounding_y", "yr[c] = oracle_bf16_rne(yv);", "yr[c] = oracle_bf16_rne((double)(float)yv);", 0),
     ("batch_stride_ignored", "return b * st[0] + f * st[1] + l * st[2];", "return f * st[1] + l * st[2];", 0),
+    ("gate_on_residual", "oracle_bf16_to_double(rr[c]) + g * oracle_bf16_to_double(xr[c])",
+     "g * oracle_bf16_to_double(rr[c]) + oracle_bf16_to_double(xr[c])", 0),
+    ("shift_with_scale_strides", "shift + row_offset(shift_st, b, f, l)", "shift + row_offset(scale_st, b, f, l)", 0),
+    ("frame_from_flat_row", "l / tokens_per_frame : 0", "row / tokens_per_frame : 0", 0),
 ]
 
 

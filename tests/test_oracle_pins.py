@@ -404,8 +404,12 @@ def test_p8_matches_torch_norms(is_rms):
 # Operand resolution: strides for broadcast, per-row, per-frame and per-batch layouts
 # --------------------------------------------------------------------------
 
-@pytest.mark.parametrize("layout", ["bcast", "row", "frame", "batch"])
-def test_operand_layouts_match_explicit_gather(layout):
+@pytest.mark.parametrize("layouts", [("bcast",) * 3, ("row",) * 3, ("frame",) * 3, ("batch",) * 3,
+                                     ("row", "frame", "bcast"), ("batch", "row", "frame"),
+                                     ("bcast", "batch", "row")], ids=lambda l: "-".join(l))
+def test_operand_layouts_match_explicit_gather(layouts):
+    # gate, scale and shift each resolved through its own strides (mixed layouts catch an
+    # operand read through another operand's strides)
     B, F, T, D = 2, 3, 4, 16
     L = F * T
     rng = np.random.default_rng(9)
@@ -413,22 +417,22 @@ def test_operand_layouts_match_explicit_gather(layout):
     def rnd(n, sd=1.0):
         return f32_to_bf16_bits_rne((sd * rng.normal(size=(n, D))).astype(np.float32))
 
-    n_stored = {"bcast": 1, "row": B * L, "frame": B * F, "batch": B}[layout]
-    st = synth.layout_strides(layout, B, L, D, F)
+    n_stored = {"bcast": 1, "row": B * L, "frame": B * F, "batch": B}
+    st = {op: synth.layout_strides(lay, B, L, D, F) for op, lay in zip(("gate", "scale", "shift"), layouts)}
     x, res = rnd(B * L), rnd(B * L)
-    gate, sc, sh = rnd(n_stored, .5), rnd(n_stored, .1), rnd(n_stored, .1)
+    gate, sc, sh = (rnd(n_stored[lay], sd) for lay, sd in zip(layouts, (.5, .1, .1)))
     row_st = (L * D, 0, D)
     got = oracle.fused_norm(B, L, D, x=x, x_st=row_st, residual=res, res_st=row_st, gate=gate,
-                            gate_st=st, scale=sc, scale_st=st, shift=sh, shift_st=st,
-                            tokens_per_frame=T if layout == "frame" else 0)
+                            gate_st=st["gate"], scale=sc, scale_st=st["scale"], shift=sh,
+                            shift_st=st["shift"], tokens_per_frame=T if "frame" in layouts else 0)
 
-    def which(b, l):   # the stored row token (b, l) reads, written out per layout
+    def which(layout, b, l):   # the stored row token (b, l) reads, written out per layout
         return {"bcast": 0, "row": b * L + l, "frame": b * F + l // T, "batch": b}[layout]
 
-    idx = np.array([which(b, l) for b in range(B) for l in range(L)])
+    idx = [np.array([which(lay, b, l) for b in range(B) for l in range(L)]) for lay in layouts]
     want = oracle.fused_norm(1, B * L, D, x=x, x_st=(0, 0, D), residual=res, res_st=(0, 0, D),
-                             gate=gate[idx], gate_st=(0, 0, D), scale=sc[idx], scale_st=(0, 0, D),
-                             shift=sh[idx], shift_st=(0, 0, D))
+                             gate=gate[idx[0]], gate_st=(0, 0, D), scale=sc[idx[1]],
+                             scale_st=(0, 0, D), shift=sh[idx[2]], shift_st=(0, 0, D))
     assert np.array_equal(got["y"].reshape(-1, D), want["y"].reshape(-1, D))
     assert np.array_equal(got["r"].reshape(-1, D), want["r"].reshape(-1, D))
 
