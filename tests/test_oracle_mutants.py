@@ -61,32 +61,48 @@ def _apply(text, old, new, occurrence):
 
 
 def _run_pins(lib_path):
-    env = dict(os.environ, ORACLE_LIB=lib_path, OMP_NUM_THREADS="4")
+    env = dict(os.environ, ORACLE_LIB=lib_path, OMP_NUM_THREADS="2")
     cmd = [sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
            os.path.join(ROOT, "tests", "test_oracle_pins.py")]
-    return subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    return subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
 
 
-def _build(tmp_path, text, name):
+def _build(directory, text, name):
     sys.path.insert(0, ROOT)
     from oracle.build import build
 
-    src = tmp_path / f"{name}.c"
-    src.write_text(text)
-    return build(str(src), str(tmp_path / f"lib{name}.so"))
+    src = os.path.join(directory, f"{name}.c")
+    with open(src, "w") as f:
+        f.write(text)
+    return build(src, os.path.join(directory, f"lib{name}.so"))
 
 
-def test_unmodified_oracle_passes_pins(tmp_path):
-    lib = _build(tmp_path, open(SRC).read(), "clean")
-    res = _run_pins(lib)
+@pytest.fixture(scope="module")
+def pin_runs(tmp_path_factory):
+    """Every mutant (and the unmodified oracle) built and run against the pins, the
+    builds and pin runs in parallel (each is its own subprocess)."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    directory = str(tmp_path_factory.mktemp("mutants"))
+    text = open(SRC).read()
+    cases = [("clean", text)] + [(name, _apply(text, old, new, occ)) for name, old, new, occ in MUTANTS]
+
+    def one(case):
+        name, src = case
+        return name, (src != text or name == "clean"), _run_pins(_build(directory, src, name))
+
+    workers = max(2, min(8, (os.cpu_count() or 2) // 2))
+    with ThreadPoolExecutor(workers) as ex:
+        return {name: (changed, res) for name, changed, res in ex.map(one, cases)}
+
+
+def test_unmodified_oracle_passes_pins(pin_runs):
+    _, res = pin_runs["clean"]
     assert res.returncode == 0, res.stdout[-2000:]
 
 
-@pytest.mark.parametrize("name,old,new,occ", MUTANTS, ids=[m[0] for m in MUTANTS])
-def test_mutant_is_caught(tmp_path, name, old, new, occ):
-    text = open(SRC).read()
-    mutated = _apply(text, old, new, occ)
-    assert mutated != text
-    lib = _build(tmp_path, mutated, name)
-    res = _run_pins(lib)
+@pytest.mark.parametrize("name", [m[0] for m in MUTANTS])
+def test_mutant_is_caught(pin_runs, name):
+    changed, res = pin_runs[name]
+    assert changed, f"mutant {name} did not change the source"
     assert res.returncode != 0, f"mutant {name} passed every pin:\n{res.stdout[-1500:]}"
