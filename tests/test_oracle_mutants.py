@@ -50,6 +50,10 @@ MUTANTS = [
      "g * oracle_bf16_to_double(rr[c]) + oracle_bf16_to_double(xr[c])", 0),
     ("shift_with_scale_strides", "shift + row_offset(shift_st, b, f, l)", "shift + row_offset(scale_st, b, f, l)", 0),
     ("frame_from_flat_row", "l / tokens_per_frame : 0", "row / tokens_per_frame : 0", 0),
+    ("layernorm_not_centred", "double n = (v[c] - mu) * rho;", "double n = v[c] * rho;", 0),
+    ("eps_as_floor", "1.0 / sqrt(second + eps)", "1.0 / sqrt(second > eps ? second : eps)", 0),
+    ("rho_in_float", "double rho = 1.0 / sqrt(second + eps);",
+     "double rho = (double)(1.0f / sqrtf((float)(second + eps)));", 0),
 ]
 
 
