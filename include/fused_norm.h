@@ -139,6 +139,10 @@ fn_status fused_norm_validate(fused_norm_t h, const fn_args* a);
  * Validate (as above), then launch the kernel on `stream`. Asynchronous: returns
  * once the launch is queued. B * L == 0 launches nothing. On FN_ERR_CUDA the CUDA
  * error code is kept per host thread (fused_norm_last_cuda_error).
+ * One kernel launch per call. Which compiled instance runs depends on the strides as
+ * well as on the handle: when scale and shift both have stride_l == 0 (broadcast, per
+ * batch or per frame) an instance that re-reads them from cache runs with more rows per
+ * SM; the results are the same bits either way.
  */
 fn_status fused_norm_launch(fused_norm_t h, const fn_args* a, fn_stream_t stream);
 
