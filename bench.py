@@ -357,7 +357,7 @@ def run_ours(args):
     # streams so copies in, compute and copies out overlap.
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, w, spec, host, d, dev, world, local, fn, torch, dist)
+        e2e = run_e2e(args, w, spec, host, d, dev, world, local, fn, torch, dist, y, r)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -395,7 +395,7 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_e2e(args, w, spec, host, d, dev, world, local, fn, torch, dist):
+def run_e2e(args, w, spec, host, d, dev, world, local, fn, torch, dist, y_ref=None, r_ref=None):
     norm = "rms" if spec.is_rms else "layer"
     rows = w.rows
     chunk = 4096
@@ -487,8 +487,33 @@ def run_e2e(args, w, spec, host, d, dev, world, local, fn, torch, dist):
     return {"value": round(world * w.algorithmic_bytes(spec) / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "ms_per_step": round(ms, 3), "steps": K, "h2d_bytes_per_step": h2d_bytes,
             "d2h_bytes_per_step": d2h_bytes,
+            "verified": _same_rows(torch, w, hy, hr, y_ref, r_ref, chunk),
             "how": "pinned host inputs copied in and outputs copied out every step, 4096-row "
                    "chunks pipelined over copy-in / compute / copy-out streams"}
+
+
+def _same_rows(torch, w, hy, hr, y_ref, r_ref, chunk):
+    """Whether the outputs copied back to the host equal, bit for bit, the device outputs of
+    the timed launches (same inputs, deterministic kernel) on sampled rows: the first and
+    last row of every 16th chunk, the first and last chunk whole, the middle row. Reports,
+    never raises: the check must not cost the benchmark its line."""
+    if y_ref is None:
+        return None
+    try:
+        rows = w.rows
+        pick = set(range(min(chunk, rows))) | set(range(max(rows - chunk, 0), rows)) | {rows // 2}
+        for c0 in range(0, rows, 16 * chunk):
+            pick |= {c0, min(rows, c0 + chunk) - 1}
+        idx = torch.tensor(sorted(pick), dtype=torch.long)
+        pairs = [(hy, y_ref)] + ([(hr, r_ref)] if hr is not None and r_ref is not None else [])
+        for host_t, dev_t in pairs:
+            a = host_t.view(-1, w.D)[idx].view(torch.int16)
+            b = dev_t.view(-1, w.D)[idx.to(dev_t.device)].cpu().view(torch.int16)
+            if not torch.equal(a, b):
+                return False
+        return True
+    except Exception as exc:  # reported, not raised
+        return f"not checked: {type(exc).__name__}: {exc}"[:200]
 
 
 # ------------------------------------------------------------------ oracle (CPU)

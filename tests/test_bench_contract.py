@@ -47,6 +47,7 @@ def test_gpu_arm_line():
     assert d["gpu_launches"] == 20
     e = d["e2e"]
     assert e["value"] > 0 and e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0
+    assert e["verified"] is True, e["verified"]      # host copies equal the device outputs
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["config"]["launch"] == "stream"
     cb = d["cpu_baseline"]
@@ -68,6 +69,7 @@ def test_gpu_arm_norm_only():
               "--rows", "4096", "--steps", "10", "--warmup", "3", "--cpu-seconds", "1"])
     assert d["config"]["spec"] == "ln_nss_now" and d["value"] > 0
     assert d["e2e"]["d2h_bytes_per_step"] == 4096 * 5120 * 2   # y only
+    assert d["e2e"]["verified"] is True, d["e2e"]["verified"]
 
 
 def test_kernel_digest_ignores_comments_only():
