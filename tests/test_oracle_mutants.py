@@ -54,6 +54,10 @@ MUTANTS = [
     ("eps_as_floor", "1.0 / sqrt(second + eps)", "1.0 / sqrt(second > eps ? second : eps)", 0),
     ("rho_in_float", "double rho = 1.0 / sqrt(second + eps);",
      "double rho = (double)(1.0f / sqrtf((float)(second + eps)));", 0),
+    ("mean_accumulated_in_float", "for (int64_t c = 0; c < D; ++c) mu += v[c];",
+     "for (int64_t c = 0; c < D; ++c) mu = (double)(float)(mu + v[c]);", 0),
+    ("variance_accumulated_in_float", "second += (v[c] - mu) * (v[c] - mu);",
+     "second = (double)(float)(second + (v[c] - mu) * (v[c] - mu));", 0),
 ]
 
 
