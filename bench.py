@@ -1,14 +1,15 @@
 """Benchmark of the fused residual / gate / norm / modulation kernel on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--rows L] [--no-e2e] [--no-cpu-baseline]
+                    [--workload NAME] [--spec NAME] [--rows L] [--graph | --flush-l2]
+                    [--no-e2e] [--no-cpu-baseline] [--e2e-steps E] [--cpu-seconds S]
 
 One step = one call of the op over the whole workload (every full tensor read or
 written once). Default workload: WAN2.2-shaped LayerNorm, B=1 L=176400 D=5120 bf16,
 gate (1,D), per-row scale/shift, no affine weight (the shape the pages' microbenchmark
 uses: sglang PR #36349, section "Microbenchmark"). Inputs are seeded synthetic
 bf16 values; they are larger than L2 (7.2 GB read per step), so no flush is needed
-between steps.
+between steps (the small L=16 workloads can flush L2 before every launch: --flush-l2).
 
 Metric: achieved HBM GB/s, counting the algorithmic bytes (each full tensor once,
 broadcast operands once), also reported as rows/s and as a fraction of the measured
