@@ -23,7 +23,7 @@ struct fused_norm_s {
   fn_config cfg;
   LaunchFn launch;            // scale or shift changes from token to token
   LaunchFn launch_cached_mod;  // scale and shift both broadcast, per batch or per frame
-  int threads;
+  int threads, threads_cached_mod;
 };
 
 namespace {
@@ -244,6 +244,8 @@ fn_status fused_norm_create(fused_norm_t* out, const fn_config* cfg) {
   h->launch = fn;
   h->launch_cached_mod = fn_cm;
   h->threads = c.D / (8 * (c.D == 5120 ? RowShape<5120>::VPT : RowShape<10240>::VPT));
+  h->threads_cached_mod =
+      c.D / (8 * (c.D == 5120 ? RowShape<5120>::kVptCachedMod : RowShape<10240>::kVptCachedMod));
   *out = h;
   return FN_OK;
 }
@@ -255,7 +257,7 @@ fn_status fused_norm_plan(fused_norm_t h, const fn_args* a, int64_t* grid, int* 
   FN_TRY(validate(h, a));
   if (!grid || !block || !smem_bytes) return FN_ERR_INVALID_ARG;
   *grid = grid_for(a->B * a->L);
-  *block = h->threads;
+  *block = (a->scale.stride_l == 0 && a->shift.stride_l == 0) ? h->threads_cached_mod : h->threads;
   *smem_bytes = 0;
   return FN_OK;
 }
@@ -266,7 +268,7 @@ fn_status fused_norm_launch(fused_norm_t h, const fn_args* a, fn_stream_t stream
   if (rows == 0) return FN_OK;
   RowParams p = make_params(h, a);
   const bool cached_mod = a->scale.stride_l == 0 && a->shift.stride_l == 0;
-  cudaError_t e = (cached_mod ? h->launch_cached_mod : h->launch)(p, grid_for(rows),
+  cudaError_t e = (cached_mod ? h->launch_cached_mod : h->launch)(p, grid_for(a->B * a->L),
                                                                   reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
     g_last_cuda_error = (int)e;

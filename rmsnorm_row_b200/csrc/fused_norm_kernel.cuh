@@ -21,13 +21,14 @@
 //     results are bitwise reproducible.
 //   * Output rounding: y is evaluated in fp32 with the fp64 statistics rounded to
 //     fp32, together with a bound on its error (8 units of fp32 roundoff times the
-//     sum of the magnitudes that enter it). When that bound does not reach the
-//     nearest bf16 rounding boundary the fp32 result rounds like the exact value;
-//     otherwise (a few in 10^4 elements) the element is recomputed in fp64 and
-//     rounded once (round-to-odd to fp32, then nearest-even to bf16). y is therefore
-//     the correctly rounded bf16 of the formula evaluated with the fp64 statistics.
-//     At D = 10240 the fp32 arithmetic runs two elements per instruction (sm_100
-//     f32x2), with results identical to the scalar form.
+//     sum of the magnitudes that enter it). The value minus the bound, rounded down,
+//     and plus the bound, rounded up, enclose the exact value; when both ends round to
+//     the same bf16 value, so does the exact value (rounding is monotone), and that is
+//     the result. Otherwise (a few in 10^4 elements) the element is recomputed in fp64
+//     and rounded once (round-to-odd to fp32, then nearest-even to bf16). y is therefore
+//     the correctly rounded bf16 of the formula evaluated with the fp64 statistics
+//     (up to the fp64 evaluation's own last-bit error). The fp32 arithmetic can run two
+//     elements per instruction (sm_100 f32x2), with results identical to the scalar form.
 //   * r is the correctly rounded bf16 of the exact residual + gate * x: one bf16x2
 //     fused multiply-add per pair computes the exact value and rounds it once.
 //   * Per-row (streamed-once) operands use evict-first loads and stores; broadcast
@@ -40,6 +41,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <type_traits>
 
 namespace fused_norm_impl {
 
@@ -81,6 +84,12 @@ __device__ __forceinline__ uint32_t word(const uint4& v, int i) {
 // element q (0..7) of a 16-byte vector of bf16, as fp32
 __device__ __forceinline__ float elem(const uint4& v, int q) {
   return (q & 1) ? hi_f(word(v, q >> 1)) : lo_f(word(v, q >> 1));
+}
+
+// Element q's value from a 16-byte vector, for a runtime q (rare paths only).
+__device__ __forceinline__ float elem_dyn(const uint4& v, int q) {
+  const uint32_t w = q < 2 ? v.x : q < 4 ? v.y : q < 6 ? v.z : v.w;
+  return (q & 1) ? hi_f(w) : lo_f(w);
 }
 
 // ---- bf16 arithmetic on packed pairs (sm_90+ bf16x2, sm_100 mixed precision) ----
@@ -172,8 +181,8 @@ __device__ __forceinline__ uint32_t y_exact(float v, float w, float b, float s, 
   return bf16_from_double(y);
 }
 
-// fp32 evaluation of y for one element, and whether it is far enough from every bf16
-// rounding boundary to be rounded as is (otherwise `near` is set).
+// fp32 evaluation of y for one element, widened to an interval [lo, hi] that holds
+// the exact value of the formula with the fp64 statistics.
 //
 // Error of the fp32 evaluation, to first order in u = 2^-24 (mu and rho are exact to
 // far better than u). With exact n* = (v - mu) rho, the eight roundings (-mu, rho,
@@ -181,14 +190,15 @@ __device__ __forceinline__ uint32_t y_exact(float v, float w, float b, float s, 
 // the final fma) give
 //   |y - y*| <= u (|1+s| |w| kappa + 7 |1+s| |n* w| + 3 |1+s| |b| + |shift|) <= 7 u P,
 //   P = |1+s| (|w| kappa + |n w| + |b|) + |shift|,  kappa = |mu| rho.
-// The test uses B = 8 u P, which also covers second-order terms and P's own rounding.
-// Rounding boundaries next to y: the midpoint D away in its bf16 interval, and, when y
-// lies in the lowest interval of a binade, one at least ulp/4 below (ulp = bf16 spacing
-// at y; |y| 2^-10 <= ulp/4). So y rounds correctly if B < min(D, |y| 2^-10).
+// The interval is y -/+ 8 u P with its ends rounded outward (down, up); 8 u instead of
+// 7 u covers second-order terms and P's own rounding. If both ends round to the same
+// bf16 value, the exact value rounds to it too (round to nearest is monotone, across
+// binade edges included); otherwise the element takes the fp64 path.
+constexpr float k8u = 4.76837158203125e-7f;  // 2^-21
+
 template <int H, bool HAS_WEIGHT, bool HAS_BIAS>
-__device__ __forceinline__ float y_fast_core(uint32_t vw, uint32_t sw, uint32_t tw, float w, float b,
-                                             const RowStats& st, bool& near) {
-  constexpr float k8u = 4.76837158203125e-7f;  // 2^-21
+__device__ __forceinline__ void y_enclose(uint32_t vw, uint32_t sw, uint32_t tw, float w, float b,
+                                          const RowStats& st, float& lo, float& hi) {
   const float n = add_bf16_f32<H>(vw, st.neg_mu32) * st.rho32;
   const float nw = HAS_WEIGHT ? n * w : n;
   const float nb = HAS_BIAS ? nw + b : nw;
@@ -197,12 +207,9 @@ __device__ __forceinline__ float y_fast_core(uint32_t vw, uint32_t sw, uint32_t 
   const float y = fmaf(nb, a, t);
   float inner = HAS_WEIGHT ? fmaf(fabsf(w), st.kappa, fabsf(nw)) : st.kappa + fabsf(nw);
   if (HAS_BIAS) inner += fabsf(b);
-  const float bound = fmaf(fabsf(a), inner, fabsf(t)) * k8u;
-  // the bf16 rounding boundary next to y: same sign and exponent, low half 0x8000
-  const float mid = __uint_as_float((__float_as_uint(y) & 0xFFFF0000u) | 0x8000u);
-  const float room = fminf(fabsf(y - mid), fabsf(y) * 9.765625e-4f);  // 2^-10
-  near |= !(room > bound);  // NaN/Inf also take the fp64 path
-  return y;
+  const float p = fmaf(fabsf(a), inner, fabsf(t));
+  lo = __fmaf_rd(p, -k8u, y);
+  hi = __fmaf_ru(p, k8u, y);
 }
 
 // ---- paired fp32 arithmetic (sm_100: two fp32 lanes per instruction, each lane
@@ -225,29 +232,29 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
-__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
 __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
   uint64_t d;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
 }
-__device__ __forceinline__ float bf16_mid(float y) {
-  return __uint_as_float((__float_as_uint(y) & 0xFFFF0000u) | 0x8000u);
+__device__ __forceinline__ uint64_t fma2_rd(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rm.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fma2_ru(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rp.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
 }
 
-// y_fast_core for both elements of one packed word (low half first): the same
+// y_enclose for both elements of one packed word (low half first): the same
 // operations in the same order, two lanes per instruction where no operand needs its
-// magnitude, so each y, bound and decision is bit-identical to the scalar path.
+// magnitude, so each y, interval and decision is bit-identical to the scalar path.
 template <bool HAS_WEIGHT, bool HAS_BIAS>
-__device__ __forceinline__ void y_fast_pair(uint32_t vw, uint32_t sw, uint32_t tw, float w0, float w1,
-                                            float b0, float b1, const RowStats& st, float& y0,
-                                            float& y1, bool& near0, bool& near1) {
-  constexpr float k8u = 4.76837158203125e-7f;  // 2^-21
-  constexpr float kEdge = 9.765625e-4f;        // 2^-10
+__device__ __forceinline__ void y_enclose_pair(uint32_t vw, uint32_t sw, uint32_t tw, float w0, float w1,
+                                               float b0, float b1, const RowStats& st, float& lo0,
+                                               float& lo1, float& hi0, float& hi1) {
   const uint64_t n = mul2(pk2(add_bf16_f32<0>(vw, st.neg_mu32), add_bf16_f32<1>(vw, st.neg_mu32)),
                           pk2(st.rho32, st.rho32));
   const uint64_t nw = HAS_WEIGHT ? mul2(n, pk2(w0, w1)) : n;
@@ -263,127 +270,80 @@ __device__ __forceinline__ void y_fast_pair(uint32_t vw, uint32_t sw, uint32_t t
     in0 += fabsf(b0);
     in1 += fabsf(b1);
   }
-  const uint64_t bound = mul2(pk2(fmaf(fabsf(a0), in0, fabsf(t0)), fmaf(fabsf(a1), in1, fabsf(t1))),
-                              pk2(k8u, k8u));
-  upk2(y, y0, y1);
-  const uint64_t dm = sub2(y, pk2(bf16_mid(y0), bf16_mid(y1)));
-  const uint64_t ye = mul2(y, pk2(kEdge, kEdge));
-  float d0, d1, e0, e1, q0, q1;
-  upk2(dm, d0, d1);
-  upk2(ye, e0, e1);
-  upk2(bound, q0, q1);
-  near0 |= !(fminf(fabsf(d0), fabsf(e0)) > q0);
-  near1 |= !(fminf(fabsf(d1), fabsf(e1)) > q1);
+  const uint64_t p = pk2(fmaf(fabsf(a0), in0, fabsf(t0)), fmaf(fabsf(a1), in1, fabsf(t1)));
+  upk2(fma2_rd(p, pk2(-k8u, -k8u), y), lo0, lo1);
+  upk2(fma2_ru(p, pk2(k8u, k8u), y), hi0, hi1);
 }
 
-// y_fast_core with bf16 weight / bias taken from packed words.
-template <int H, bool HAS_WEIGHT, bool HAS_BIAS>
-__device__ __forceinline__ float y_fast(uint32_t vw, uint32_t sw, uint32_t tw, uint32_t ww,
-                                        uint32_t bw, const RowStats& st, bool& near) {
-  return y_fast_core<H, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, H ? hi_f(ww) : lo_f(ww),
-                                              H ? hi_f(bw) : lo_f(bw), st, near);
-}
-
-// Element q's value from a 16-byte vector, for a runtime q (rare paths only).
-__device__ __forceinline__ float elem_dyn(const uint4& v, int q) {
-  const uint32_t w = q < 2 ? v.x : q < 4 ? v.y : q < 6 ? v.z : v.w;
-  return (q & 1) ? hi_f(w) : lo_f(w);
-}
-
-// One 16-byte vector of y: the fp32 fast path for all eight elements, then (rarely) the
-// fp64 path for the elements whose fast value came near a rounding boundary.
-template <bool PAIRED, bool HAS_WEIGHT, bool HAS_BIAS>
-__device__ __forceinline__ uint4 output_vec(const uint4& v, const uint4& sv, const uint4& tv,
-                                            const uint4& wv, const uint4& bv, const RowStats& st) {
-  uint32_t o[4];
-  uint32_t near_mask = 0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t vw = word(v, i), sw = word(sv, i), tw = word(tv, i);
-    const uint32_t ww = word(wv, i), bw = word(bv, i);
-    bool n0 = false, n1 = false;
-    float y0, y1;
-    if (PAIRED) {
-      y_fast_pair<HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, lo_f(ww), hi_f(ww), lo_f(bw), hi_f(bw), st, y0, y1,
-                                        n0, n1);
-    } else {
-      y0 = y_fast<0, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, ww, bw, st, n0);
-      y1 = y_fast<1, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, ww, bw, st, n1);
-    }
-    o[i] = pack_rn(y0, y1);
-    near_mask |= (n0 ? 1u : 0u) << (2 * i);
-    near_mask |= (n1 ? 2u : 0u) << (2 * i);
-  }
-  uint4 out = make_uint4(o[0], o[1], o[2], o[3]);
-#pragma unroll 1
-  while (near_mask) {  // rare
-    const int q = __ffs(near_mask) - 1;
-    near_mask &= near_mask - 1;
-    const uint32_t bits = y_exact<HAS_WEIGHT, HAS_BIAS>(
-        elem_dyn(v, q), HAS_WEIGHT ? elem_dyn(wv, q) : 1.0f, HAS_BIAS ? elem_dyn(bv, q) : 0.0f,
-        elem_dyn(sv, q), elem_dyn(tv, q), st.mu, st.rho);
-    const uint32_t put = (q & 1) ? (bits << 16) : bits;
-    const uint32_t keep = (q & 1) ? 0x0000FFFFu : 0xFFFF0000u;
-    const int i = q >> 1;
-    out.x = i == 0 ? ((out.x & keep) | put) : out.x;
-    out.y = i == 1 ? ((out.y & keep) | put) : out.y;
-    out.z = i == 2 ? ((out.z & keep) | put) : out.z;
-    out.w = i == 3 ? ((out.w & keep) | put) : out.w;
-  }
-  return out;
-}
-
-// fp32 affine parameters (w, b as given, 8 per vector: two 16-byte loads each).
-struct Affine8 {
+// Affine parameters of 8 consecutive channels: fp32 as given (two 16-byte loads) or
+// bf16 (one 16-byte load, each value widened exactly where it is used).
+struct AffineF32 {
   float v[8];
+  __device__ __forceinline__ float operator[](int q) const { return v[q]; }
+  __device__ __forceinline__ float at(int q) const {  // runtime q (rare paths only)
+    return q == 0 ? v[0] : q == 1 ? v[1] : q == 2 ? v[2] : q == 3 ? v[3]
+         : q == 4 ? v[4] : q == 5 ? v[5] : q == 6 ? v[6] : v[7];
+  }
+  static __device__ __forceinline__ AffineF32 load(const void* p, int j) {
+    const float4* f = reinterpret_cast<const float4*>(p) + 2 * j;
+    const float4 a = __ldg(f), c = __ldg(f + 1);
+    return AffineF32{{a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w}};
+  }
+  static __device__ __forceinline__ AffineF32 fill(float x) { return AffineF32{{x, x, x, x, x, x, x, x}}; }
 };
-__device__ __forceinline__ Affine8 load_affine_f32(const void* p, int j) {
-  const float4* f = reinterpret_cast<const float4*>(p) + 2 * j;
-  const float4 a = __ldg(f), c = __ldg(f + 1);
-  return Affine8{{a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w}};
-}
-__device__ __forceinline__ float sel8(const Affine8& a, int q) {
-  return q == 0 ? a.v[0] : q == 1 ? a.v[1] : q == 2 ? a.v[2] : q == 3 ? a.v[3]
-       : q == 4 ? a.v[4] : q == 5 ? a.v[5] : q == 6 ? a.v[6] : a.v[7];
-}
+struct AffineBF16 {
+  uint4 u;
+  __device__ __forceinline__ float operator[](int q) const { return elem(u, q); }
+  __device__ __forceinline__ float at(int q) const { return elem_dyn(u, q); }
+  static __device__ __forceinline__ AffineBF16 load(const void* p, int j) {
+    return AffineBF16{__ldg(reinterpret_cast<const uint4*>(p) + j)};
+  }
+  static __device__ __forceinline__ AffineBF16 fill(float x) {
+    const uint32_t h = __float_as_uint(x) >> 16;  // 0 and 1 are exact in bf16
+    return AffineBF16{make_uint4(h * 0x10001u, h * 0x10001u, h * 0x10001u, h * 0x10001u)};
+  }
+};
 
-// As output_vec, with fp32 weight / bias.
-template <bool PAIRED, bool HAS_WEIGHT, bool HAS_BIAS>
-__device__ __forceinline__ uint4 output_vec_f32(const uint4& v, const uint4& sv, const uint4& tv,
-                                                const Affine8& wf, const Affine8& bf,
-                                                const RowStats& st) {
-  uint32_t o[4];
-  uint32_t near_mask = 0;
+// One 16-byte vector of y: the fp32 interval for all eight elements, packed to bf16 at
+// both ends; then (rarely) the fp64 path for the elements whose ends differ.
+template <bool PAIRED, bool HAS_WEIGHT, bool HAS_BIAS, class Affine>
+__device__ __forceinline__ uint4 output_vec(const uint4& v, const uint4& sv, const uint4& tv,
+                                            const Affine& wf, const Affine& bf, const RowStats& st) {
+  uint32_t o[4], d[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const uint32_t vw = word(v, i), sw = word(sv, i), tw = word(tv, i);
-    bool n0 = false, n1 = false;
-    float y0, y1;
+    const int e = 2 * i, f = 2 * i + 1;
+    float lo0, lo1, hi0, hi1;
     if (PAIRED) {
-      y_fast_pair<HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, wf.v[2 * i], wf.v[2 * i + 1], bf.v[2 * i],
-                                        bf.v[2 * i + 1], st, y0, y1, n0, n1);
+      y_enclose_pair<HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, wf[e], wf[f], bf[e], bf[f], st, lo0, lo1, hi0, hi1);
     } else {
-      y0 = y_fast_core<0, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, wf.v[2 * i], bf.v[2 * i], st, n0);
-      y1 = y_fast_core<1, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, wf.v[2 * i + 1], bf.v[2 * i + 1], st, n1);
+      y_enclose<0, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, wf[e], bf[e], st, lo0, hi0);
+      y_enclose<1, HAS_WEIGHT, HAS_BIAS>(vw, sw, tw, wf[f], bf[f], st, lo1, hi1);
     }
-    o[i] = pack_rn(y0, y1);
-    near_mask |= (n0 ? 1u : 0u) << (2 * i);
-    near_mask |= (n1 ? 2u : 0u) << (2 * i);
+    o[i] = pack_rn(hi0, hi1);
+    d[i] = pack_rn(lo0, lo1) ^ o[i];
   }
   uint4 out = make_uint4(o[0], o[1], o[2], o[3]);
+  if ((d[0] | d[1]) | (d[2] | d[3])) {  // rare
+    uint32_t near_mask = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      near_mask |= ((d[i] & 0xFFFFu) ? 1u : 0u) << (2 * i) | ((d[i] >> 16) ? 2u : 0u) << (2 * i);
 #pragma unroll 1
-  while (near_mask) {  // rare
-    const int q = __ffs(near_mask) - 1;
-    near_mask &= near_mask - 1;
-    const uint32_t bits = y_exact<HAS_WEIGHT, HAS_BIAS>(elem_dyn(v, q), sel8(wf, q), sel8(bf, q),
-                                                        elem_dyn(sv, q), elem_dyn(tv, q), st.mu, st.rho);
-    const uint32_t put = (q & 1) ? (bits << 16) : bits;
-    const uint32_t keep = (q & 1) ? 0x0000FFFFu : 0xFFFF0000u;
-    const int i = q >> 1;
-    out.x = i == 0 ? ((out.x & keep) | put) : out.x;
-    out.y = i == 1 ? ((out.y & keep) | put) : out.y;
-    out.z = i == 2 ? ((out.z & keep) | put) : out.z;
-    out.w = i == 3 ? ((out.w & keep) | put) : out.w;
+    while (near_mask) {
+      const int q = __ffs(near_mask) - 1;
+      near_mask &= near_mask - 1;
+      const uint32_t bits = y_exact<HAS_WEIGHT, HAS_BIAS>(elem_dyn(v, q), wf.at(q), bf.at(q),
+                                                          elem_dyn(sv, q), elem_dyn(tv, q), st.mu, st.rho);
+      const uint32_t put = (q & 1) ? (bits << 16) : bits;
+      const uint32_t keep = (q & 1) ? 0x0000FFFFu : 0xFFFF0000u;
+      const int i = q >> 1;
+      out.x = i == 0 ? ((out.x & keep) | put) : out.x;
+      out.y = i == 1 ? ((out.y & keep) | put) : out.y;
+      out.z = i == 2 ? ((out.z & keep) | put) : out.z;
+      out.w = i == 3 ? ((out.w & keep) | put) : out.w;
+    }
   }
   return out;
 }
@@ -404,23 +364,29 @@ template <int D> struct RowShape;
 #ifndef FN_MINB_10240
 #define FN_MINB_10240 2
 #endif
-// 1: y's fp32 arithmetic in paired (f32x2) instructions. Bit-identical either way; it
-// cuts ~6% of the instructions but lengthens each thread's dependency chains. Measured
-// on B200: ~4% faster at D = 10240 (two CTAs per SM, issue-bound with weight), neutral
-// to mixed at D = 5120 and slower there when launches run serialised.
 // CTAs per SM for the instances whose scale and shift are broadcast or per frame: they
 // fetch scale and shift from L1 as each vector is used instead of holding them across
 // the statistics, which frees registers for more rows per SM (measured on B200: frame
 // gate, broadcast fused and norm-only shapes 2-5% faster than with the streamed
-// instances; 7 CTAs at D = 5120 is slower again).
+// instances; 7 CTAs at D = 5120 is slower again for the fused ones).
+#ifndef FN_VPT_CM_5120
+#define FN_VPT_CM_5120 FN_VPT_5120
+#endif
+#ifndef FN_VPT_CM_10240
+#define FN_VPT_CM_10240 FN_VPT_10240
+#endif
 #ifndef FN_MINB_CM_5120
 #define FN_MINB_CM_5120 6
 #endif
 #ifndef FN_MINB_CM_10240
 #define FN_MINB_CM_10240 3
 #endif
+// 1: y's fp32 arithmetic in paired (f32x2) instructions where no operand needs its
+// magnitude. Bit-identical either way; it cuts the instructions per element. Measured on
+// B200 with the interval check: 1-3% faster on the broadcast, frame-gate, norm-only
+// and D = 10240 shapes, neutral on the WAN2.2 shape.
 #ifndef FN_PAIRED_5120
-#define FN_PAIRED_5120 0
+#define FN_PAIRED_5120 1
 #endif
 #ifndef FN_PAIRED_10240
 #define FN_PAIRED_10240 1
@@ -431,21 +397,41 @@ template <int D> struct RowShape;
 #ifndef FN_EARLY_MODULATION_LOADS
 #define FN_EARLY_MODULATION_LOADS 0
 #endif
+// Norm-only with broadcast / per-frame scale and shift reads one tensor and writes one
+// per row, so its per-element arithmetic, not HBM, sets its pace: those instances run
+// 7 CTAs per SM (72 registers), one more than the other broadcast instances, and sum
+// squares with two fused multiply-adds per pair (one instruction fewer; where the
+// other instances' register budgets leave no room for it, they keep the product form).
+#ifndef FN_MINB_NSS_5120
+#define FN_MINB_NSS_5120 7
+#endif
+#ifndef FN_MINB_NSS_10240
+#define FN_MINB_NSS_10240 FN_MINB_CM_10240
+#endif
 template <> struct RowShape<5120> {
   static constexpr int VPT = FN_VPT_5120, kMinBlocks = FN_MINB_5120;
-  static constexpr int kMinBlocksCachedMod = FN_MINB_CM_5120;
+  static constexpr int kMinBlocksCachedMod = FN_MINB_CM_5120, kVptCachedMod = FN_VPT_CM_5120;
+  static constexpr int kMinBlocksNss = FN_MINB_NSS_5120;
   static constexpr bool kPaired = FN_PAIRED_5120 != 0;
 };
 template <> struct RowShape<10240> {
   static constexpr int VPT = FN_VPT_10240, kMinBlocks = FN_MINB_10240;
-  static constexpr int kMinBlocksCachedMod = FN_MINB_CM_10240;
+  static constexpr int kMinBlocksCachedMod = FN_MINB_CM_10240, kVptCachedMod = FN_VPT_CM_10240;
+  static constexpr int kMinBlocksNss = FN_MINB_NSS_10240;
   static constexpr bool kPaired = FN_PAIRED_10240 != 0;
 };
 
+// CTAs per SM an instance's register budget is sized for.
+template <int D, bool NORM_ONLY, bool CACHED_MOD>
+constexpr int min_blocks() {
+  return (NORM_ONLY && CACHED_MOD) ? RowShape<D>::kMinBlocksNss
+         : CACHED_MOD              ? RowShape<D>::kMinBlocksCachedMod
+                                   : RowShape<D>::kMinBlocks;
+}
+
 template <int D, int VPT, bool IS_RMS, bool NORM_ONLY, bool HAS_GATE, bool HAS_WEIGHT, bool HAS_BIAS,
           bool AFFINE_F32, bool CACHED_MOD>
-__global__ void __launch_bounds__(D / (8 * VPT), CACHED_MOD ? RowShape<D>::kMinBlocksCachedMod
-                                                            : RowShape<D>::kMinBlocks)
+__global__ void __launch_bounds__(D / (8 * VPT), (min_blocks<D, NORM_ONLY, CACHED_MOD>()))
 fused_norm_rows(const RowParams p) {
   constexpr int T = D / (8 * VPT);
   constexpr int W = T / 32;
@@ -472,6 +458,7 @@ fused_norm_rows(const RowParams p) {
     // a load written after a store waits for the store's issue, since the compiler
     // cannot rule out aliasing.
     uint4 xv[VPT], rv[VPT], gv[VPT], sv[VPT], tv[VPT];
+#pragma unroll
 #pragma unroll
     for (int k = 0; k < VPT; ++k) xv[k] = load_vec(xr, tid + k * T, p.stream_mask & kX);
     if (!NORM_ONLY) {
@@ -524,7 +511,10 @@ fused_norm_rows(const RowParams p) {
       for (int i = 0; i < 4; ++i) {
         const double a = bf16_f64<0>(word(v[k], i)), c = bf16_f64<1>(word(v[k], i));
         if (!IS_RMS) a1[i] += a + c;                 // a + c exact: two bf16 values
-        a2[i] += fma(a, a, c * c);                   // c * c exact (16-bit significand)
+        if (NORM_ONLY)
+          a2[i] = fma(c, c, fma(a, a, a2[i]));       // squares of bf16 values: exact
+        else
+          a2[i] += fma(a, a, c * c);                 // c * c exact (16-bit significand)
       }
     double s1 = (a1[0] + a1[1]) + (a1[2] + a1[3]);
     double s2 = (a2[0] + a2[1]) + (a2[2] + a2[3]);
@@ -596,34 +586,32 @@ fused_norm_rows(const RowParams p) {
         sv[k] = __ldg(reinterpret_cast<const uint4*>(sr) + j);
         tv[k] = __ldg(reinterpret_cast<const uint4*>(tr) + j);
       }
-      if (AFFINE_F32) {
-        Affine8 wf{{1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f}}, bf{{0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}};
-        if (HAS_WEIGHT) wf = load_affine_f32(p.weight, j);
-        if (HAS_BIAS) bf = load_affine_f32(p.bias, j);
-        __stcs(yo + j, output_vec_f32<RowShape<D>::kPaired, HAS_WEIGHT, HAS_BIAS>(v[k], sv[k], tv[k], wf, bf, st));
-      } else {
-        uint4 wv = make_uint4(0, 0, 0, 0), bv = make_uint4(0, 0, 0, 0);
-        if (HAS_WEIGHT) wv = __ldg(reinterpret_cast<const uint4*>(p.weight) + j);
-        if (HAS_BIAS) bv = __ldg(reinterpret_cast<const uint4*>(p.bias) + j);
-        __stcs(yo + j, output_vec<RowShape<D>::kPaired, HAS_WEIGHT, HAS_BIAS>(v[k], sv[k], tv[k], wv, bv, st));
-      }
+      using Affine = typename std::conditional<AFFINE_F32, AffineF32, AffineBF16>::type;
+      const Affine wf = HAS_WEIGHT ? Affine::load(p.weight, j) : Affine::fill(1.0f);
+      const Affine bf = HAS_BIAS ? Affine::load(p.bias, j) : Affine::fill(0.0f);
+      __stcs(yo + j, output_vec<RowShape<D>::kPaired, HAS_WEIGHT, HAS_BIAS>(v[k], sv[k], tv[k], wf, bf, st));
     }
   }
 }
 
+// Launches one instance and returns the status of this launch alone (the value the
+// runtime returns for it; no earlier error is read or cleared).
 template <int D, int VPT, bool IS_RMS, bool NORM_ONLY, bool HAS_GATE, bool HAS_WEIGHT, bool HAS_BIAS,
           bool AFFINE_F32, bool CACHED_MOD>
 cudaError_t launch_rows(const RowParams& p, int64_t grid, cudaStream_t stream) {
-  constexpr int T = D / (8 * VPT);
-  fused_norm_rows<D, VPT, IS_RMS, NORM_ONLY, HAS_GATE, HAS_WEIGHT, HAS_BIAS, AFFINE_F32, CACHED_MOD>
-      <<<(unsigned)grid, T, 0, stream>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(D / (8 * VPT), 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  return cudaLaunchKernelEx(
+      &cfg, fused_norm_rows<D, VPT, IS_RMS, NORM_ONLY, HAS_GATE, HAS_WEIGHT, HAS_BIAS, AFFINE_F32, CACHED_MOD>, p);
 }
 
 // Launcher for one (norm_only, gate, modulation caching) group: the affine combinations.
 template <int D, bool RMS, bool NO, bool G, bool CM>
 LaunchFn pick_affine(bool w, bool b, bool f32) {
-  constexpr int V = RowShape<D>::VPT;
+  constexpr int V = CM ? RowShape<D>::kVptCachedMod : RowShape<D>::VPT;
   if (!w && !b) return &launch_rows<D, V, RMS, NO, G, false, false, false, CM>;
   if (f32) {
     if (w && b) return &launch_rows<D, V, RMS, NO, G, true, true, true, CM>;

@@ -1,15 +1,17 @@
-"""The kernel's rounding-margin rule, emulated on the CPU with exact IEEE arithmetic.
+"""The kernel's rounding rule for y, emulated on the CPU with exact IEEE arithmetic.
 
 The kernel evaluates y = n (1 + scale) + shift in fp32 with the fp64 row statistics
-rounded to fp32, and rounds that fp32 value to bf16 only when a bound B = 8 u P on its
-error (u = 2^-24, P = |1+s| (|w| kappa + |n w| + |b|) + |shift|, kappa = |mean| rho) stays
-below the distance to the nearest bf16 rounding boundary, min(|y - mid|, |y| 2^-10);
-every other element is recomputed in fp64. This test replays those fp32 operations one by
-one (numpy float32 arithmetic rounds each operation to nearest, fused multiply-adds are
-done exactly and rounded once) and checks, over rows built to be hard (means far above
-the spread, tiny and huge spreads, shift nearly cancelling n (1 + scale)), that every
-element the rule lets through rounds exactly like the fp64 evaluation of the formula
-(round to odd into fp32, then to nearest even), as the fallback path computes it.
+rounded to fp32, together with a bound B = 8 u P on its error (u = 2^-24,
+P = |1+s| (|w| kappa + |n w| + |b|) + |shift|, kappa = |mean| rho). It widens y to the
+interval [RD(y - B), RU(y + B)] (ends rounded down and up) and takes the bf16 rounding
+of the upper end when both ends round to the same bf16 value; every other element is
+recomputed in fp64. This test replays those fp32 operations one by one (numpy float32
+arithmetic rounds each operation to nearest; fused multiply-adds are done exactly and
+rounded once, to nearest or in the stated direction) and checks, over rows built to be
+hard (means far above the spread, tiny and huge spreads, shift nearly cancelling
+n (1 + scale)), that every element the rule lets through rounds exactly like the fp64
+evaluation of the formula (round to odd into fp32, then to nearest even), as the
+fallback path computes it.
 
 It exercises the design of the check, not the compiled kernel (the GPU parity tests do
 that); it shares nothing with the oracle.
@@ -43,14 +45,30 @@ def _f32_round_odd_then_f32(x: np.ndarray, err: np.ndarray) -> np.ndarray:
     return bits.view(np.float64).astype(np.float32)
 
 
-def _fma32(a, b, c) -> np.ndarray:
-    """fmaf: a * b + c for float32 operands with a single rounding to float32."""
+def _fma_exact(a, b, c):
+    """a * b + c for float32 operands as (RN64 value, exact remainder)."""
     p = a.astype(np.float64) * b.astype(np.float64)      # exact: 24 + 24 bits
     c64 = c.astype(np.float64)
     s = p + c64                                          # TwoSum: exact remainder
     bp = s - c64
     err = (p - bp) + (c64 - (s - bp))
-    return _f32_round_odd_then_f32(s, err)
+    return s, err
+
+
+def _fma32(a, b, c) -> np.ndarray:
+    """fmaf: a * b + c for float32 operands with a single rounding to nearest float32."""
+    return _f32_round_odd_then_f32(*_fma_exact(a, b, c))
+
+
+def _fma32_directed(a, b, c, up: bool) -> np.ndarray:
+    """fmaf with one rounding toward +inf (up) or -inf: __fmaf_ru / __fmaf_rd."""
+    s, err = _fma_exact(a, b, c)
+    f = s.astype(np.float32)
+    diff = s - f.astype(np.float64)                      # exact (f is within an fp32 ulp of s)
+    sign = np.where(diff != 0, np.sign(diff), np.sign(err))   # sign of exact - f
+    if up:
+        return np.where(sign > 0, np.nextafter(f, np.float32(np.inf)), f).astype(np.float32)
+    return np.where(sign < 0, np.nextafter(f, np.float32(-np.inf)), f).astype(np.float32)
 
 
 def _bf16_from_double(v: np.ndarray) -> np.ndarray:
@@ -61,8 +79,9 @@ def _bf16_from_double(v: np.ndarray) -> np.ndarray:
     return _bf16_rne(_f32_round_odd_then_f32(f64, v - f64))
 
 
-def _fast_path(v, s, t, w, b, mu, rho):
-    """The kernel's fp32 evaluation of y and its rounding-margin decision."""
+def _fast_path(v, s, t, w, b, mu, rho, k=F32(2.0 ** -21)):
+    """The kernel's fp32 evaluation of y, its interval and its decision: returns the
+    bf16 result of the fast path and whether the element goes to the fp64 path."""
     neg_mu = F32(-mu)
     rho32 = F32(rho)
     kappa = F32(abs(neg_mu) * rho32)
@@ -78,11 +97,11 @@ def _fast_path(v, s, t, w, b, mu, rho):
         inner = kappa + np.abs(nw)
     if b is not None:
         inner = inner + np.abs(b.astype(F32))
-    bound = _fma32(np.abs(a), inner, np.abs(t32)) * F32(2.0 ** -21)
-    mid = ((y.view(np.uint32) & np.uint32(0xFFFF0000)) | np.uint32(0x8000)).view(np.float32)
-    room = np.minimum(np.abs(y - mid), np.abs(y) * F32(2.0 ** -10))
-    near = ~(room > bound)
-    return y, near
+    p = _fma32(np.abs(a), inner, np.abs(t32))
+    lo = _fma32_directed(p, np.full_like(p, -k), y, up=False)
+    hi = _fma32_directed(p, np.full_like(p, k), y, up=True)
+    out = _bf16_rne(hi)
+    return out, _bf16_rne(lo) != out
 
 
 def _fp64_formula(v, s, t, w, b, mu, rho):
@@ -136,17 +155,29 @@ def test_fma_emulation_rounds_once():
     assert _fma32(c, np.array([3.0], dtype=np.float32), one)[0] == np.float32(1 + 2.0 ** -22)
 
 
-def test_margin_rule_never_lets_a_misrounding_through():
+def test_directed_fma_emulation():
+    # 1 + 2^-30: rounds down to 1, up to 1 + 2^-23; an exact result stays put
+    one = np.array([1.0], dtype=np.float32)
+    tiny = np.array([2.0 ** -30], dtype=np.float32)
+    assert _fma32_directed(tiny, one, one, up=False)[0] == np.float32(1.0)
+    assert _fma32_directed(tiny, one, one, up=True)[0] == np.float32(1 + 2.0 ** -23)
+    assert _fma32_directed(-tiny, one, one, up=False)[0] == np.float32(1 - 2.0 ** -24)
+    assert _fma32_directed(-tiny, one, one, up=True)[0] == np.float32(1.0)
+    half = np.array([0.5], dtype=np.float32)
+    for up in (False, True):
+        assert _fma32_directed(half, half, one, up=up)[0] == np.float32(1.25)
+
+
+def test_interval_rule_never_lets_a_misrounding_through():
     rng = np.random.default_rng(20260)
     D = 4096
     total = {"centred": 0, "offset": 0, "cancel": 0}
     flagged = dict(total)
     for v, s, t, w, b, mu, rho, kind in _rows(rng, 300, D):
-        y, near = _fast_path(v, s, t, w, b, mu, rho)
+        fast, near = _fast_path(v, s, t, w, b, mu, rho)
         ok = ~near
-        fast = _bf16_rne(y[ok])
         want = _bf16_from_double(_fp64_formula(v, s, t, w, b, mu, rho)[ok])
-        bad = np.flatnonzero(fast != want)
+        bad = np.flatnonzero(fast[ok] != want)
         assert bad.size == 0, (f"fast path misrounds {bad.size} elements, e.g. v={v[ok][bad[0]]!r} "
                                f"s={s[ok][bad[0]]!r} t={t[ok][bad[0]]!r}")
         total[kind] += D
@@ -157,24 +188,15 @@ def test_margin_rule_never_lets_a_misrounding_through():
     assert flagged["centred"] / total["centred"] < 2e-3, flagged["centred"] / total["centred"]
 
 
-def test_margin_rule_detects_a_tight_bound():
+def test_interval_rule_detects_a_tight_bound():
     # with the bound divided by 64 the rule must let misroundings through on the same
     # rows (the check above would catch a bound that is too small)
     rng = np.random.default_rng(20260)
     D = 4096
     misrounded = 0
     for v, s, t, w, b, mu, rho, _ in _rows(rng, 60, D):
-        neg_mu = F32(-mu)
-        rho32 = F32(rho)
-        n = (v.astype(F32) + neg_mu) * rho32
-        nw = n * w.astype(F32) if w is not None else n
-        nb = nw + b.astype(F32) if b is not None else nw
-        a = s.astype(F32) + F32(1)
-        y = _fma32(nb, a, t.astype(F32))
-        mid = ((y.view(np.uint32) & np.uint32(0xFFFF0000)) | np.uint32(0x8000)).view(np.float32)
-        room = np.minimum(np.abs(y - mid), np.abs(y) * F32(2.0 ** -10))
-        loose = room > F32(2.0 ** -27) * (np.abs(a) * np.abs(nw) + np.abs(t.astype(F32)))
-        fast = _bf16_rne(y[loose])
-        want = _bf16_from_double(_fp64_formula(v, s, t, w, b, mu, rho)[loose])
-        misrounded += int((fast != want).sum())
+        fast, near = _fast_path(v, s, t, w, b, mu, rho, k=F32(2.0 ** -27))
+        ok = ~near
+        want = _bf16_from_double(_fp64_formula(v, s, t, w, b, mu, rho)[ok])
+        misrounded += int((fast[ok] != want).sum())
     assert misrounded > 0
