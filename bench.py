@@ -13,9 +13,13 @@ between steps (the small L=16 workloads can flush L2 before every launch: --flus
 
 Metric: achieved HBM GB/s, counting the algorithmic bytes (each full tensor once,
 broadcast operands once), also reported as rows/s and as a fraction of the measured
-HBM copy bandwidth. Multi-GPU: one process per GPU (torchrun); each rank runs its own
-full-size problem (rows are independent, nothing is exchanged), value = all ranks'
-bytes / max-over-ranks time (weak scaling).
+HBM copy bandwidth. Multi-GPU: one process per GPU. `python bench.py --gpus N` starts
+the N ranks itself (under torch.distributed.run, on 127.0.0.1); started by torchrun
+instead, it uses the ranks it is given. Each rank runs its own full-size problem (rows
+are independent, nothing is exchanged), value = all ranks' bytes / max-over-ranks time
+(weak scaling). With several ranks the pinned host buffers of the end-to-end number are
+one copy per node in shared memory (the ranks run the same seeded problem), not one per
+rank.
 
 --impl reference times the fp64 CPU oracle (the only other implementation that
 exists) on the host cores, on bounded samples of the same workload.
@@ -160,6 +164,16 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def physical_gpus(n_local):
+    """nvidia-smi ids of the first n_local visible GPUs (CUDA_VISIBLE_DEVICES may
+    renumber or hide devices)."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").strip()
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        return ids[:n_local]
+    return [str(i) for i in range(n_local)]
+
+
 class ClockSampler:
     """nvidia-smi clock and throttle-reason samples while the timed region runs."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -240,7 +254,8 @@ def run_ours(args):
     norm = "rms" if spec.is_rms else "layer"
 
     # Inputs: generated into pinned host buffers (these are also the e2e host inputs),
-    # then copied to the device once.
+    # then copied to the device once. Several ranks share one copy per node.
+    bufs = cuda_host_buffers(torch, dist, world, local, dev)
     host = {}
     for name in ("x", "residual", "gate", "scale", "shift", "weight", "bias"):
         if name == "gate" and not spec.has_gate or name == "weight" and not spec.has_weight \
@@ -248,8 +263,7 @@ def run_ours(args):
                 or name in ("residual", "gate") and spec.norm_only:
             continue
         n = 1 if name in ("weight", "bias") else w.stored_rows(name)
-        t = torch.empty((n, w.D), dtype=torch.int16, pin_memory=True)
-        w.generate(name, out=t.numpy().view(np.uint16))
+        t = bufs.get(f"in_{name}", n * w.D, lambda a, name=name: w.generate(name, out=a.reshape(-1, w.D)))
         host[name] = t.view(torch.bfloat16).view(synth.device.operand_view_shape(w, name))
     d = {k: v.to(dev) for k, v in host.items()}
     y = torch.empty((w.B, w.L, w.D), dtype=torch.bfloat16, device=dev)
@@ -287,7 +301,8 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
 
     # rank 0 samples every GPU of this node that the job uses
-    sampler = ClockSampler(list(range(world))) if rank == 0 else None
+    local_world = int(os.environ.get("LOCAL_WORLD_SIZE", str(world)))
+    sampler = ClockSampler(physical_gpus(local_world)) if rank == 0 else None
     if sampler:
         sampler.start()
         t_end = time.time() + 1.0       # keep the GPU busy while nvidia-smi starts
@@ -358,7 +373,8 @@ def run_ours(args):
     # streams so copies in, compute and copies out overlap.
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, w, spec, host, d, dev, world, local, fn, torch, dist, y, r)
+        e2e = run_e2e(args, w, spec, host, d, dev, world, local, fn, torch, dist, y, r, bufs)
+        e2e["host_buffers"] = bufs.kind
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -392,16 +408,104 @@ def run_ours(args):
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
+    bufs.close()
     if world > 1:
         dist.destroy_process_group()
 
 
-def run_e2e(args, w, spec, host, d, dev, world, local, fn, torch, dist, y_ref=None, r_ref=None):
+class HostBuffers:
+    """Pinned host buffers (int16 elements). One rank: private pinned tensors. Several
+    ranks on one node: one copy per node in POSIX shared memory, created and filled by
+    local rank 0 and registered as pinned memory by every rank (all ranks run the same
+    seeded problem, so they read the same inputs and write the same output bytes).
+    Falls back to private buffers when /dev/shm cannot hold them.
+
+    barrier() and all_min(flag) are the job's collectives; pin(ptr, nbytes) -> bool and
+    unpin(ptr) register host memory with the GPU driver."""
+
+    def __init__(self, torch, world, local, run_id, barrier, all_min, pin, unpin, shm="/dev/shm"):
+        self.torch, self.world, self.local, self.run = torch, world, local, run_id
+        self.barrier, self.all_min, self.pin, self.unpin, self.shm = barrier, all_min, pin, unpin, shm
+        self.kind = "private pinned (one rank)" if world == 1 else "node-shared pinned"
+        self.maps, self.registered, self.paths = [], [], []
+
+    def get(self, tag, n, fill=None):
+        torch = self.torch
+        if self.world == 1 or not self.kind.startswith("node-shared"):
+            t = torch.empty(n, dtype=torch.int16, pin_memory=torch.cuda.is_available())
+            if fill is not None:
+                fill(t.numpy().view(np.uint16))
+            return t
+        import mmap
+        path = os.path.join(self.shm, f"fused_norm_bench_{self.run}_{tag}")
+        nbytes = n * 2
+        ok = True
+        if self.local == 0:
+            try:
+                st = os.statvfs(self.shm)
+                ok = st.f_bavail * st.f_frsize > nbytes + (256 << 20)
+            except OSError:
+                ok = False
+        if not self.all_min(ok):
+            self.kind = "private pinned (shared memory too small for a node-shared copy)"
+            return self.get(tag, n, fill)
+        if self.local == 0:
+            fd = os.open(path, os.O_CREAT | os.O_EXCL | os.O_RDWR, 0o600)
+            os.ftruncate(fd, nbytes)
+            mm = mmap.mmap(fd, nbytes)
+            os.close(fd)
+            self.paths.append(path)
+            if fill is not None:
+                fill(np.frombuffer(mm, dtype=np.uint16))
+        self.barrier()
+        if self.local != 0:
+            fd = os.open(path, os.O_RDWR)
+            mm = mmap.mmap(fd, nbytes)
+            os.close(fd)
+        self.maps.append(mm)
+        t = torch.from_numpy(np.frombuffer(mm, dtype=np.int16))
+        if self.pin(t.data_ptr(), nbytes):
+            self.registered.append(t.data_ptr())
+        else:
+            self.kind = "node-shared (pinning refused: pageable copies)"
+        self.barrier()
+        if self.local == 0:
+            os.unlink(path)                  # every rank has mapped it; the mappings stay valid
+            self.paths.remove(path)
+        return t
+
+    def close(self):
+        for ptr in self.registered:
+            self.unpin(ptr)
+        self.registered = []
+        for path in self.paths:
+            try:
+                os.unlink(path)
+            except OSError:
+                pass
+
+
+def cuda_host_buffers(torch, dist, world, local, dev):
+    """HostBuffers wired to NCCL collectives and cudaHostRegister."""
+    def all_min(flag):
+        t = torch.tensor([1 if flag else 0], dtype=torch.int32, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MIN)
+        return bool(t.item())
+    rt = torch.cuda.cudart()
+    return HostBuffers(torch, world, local,
+                       os.environ.get("TORCHELASTIC_RUN_ID") or os.environ.get("MASTER_PORT", "0"),
+                       barrier=lambda: dist.barrier(device_ids=[local]), all_min=all_min,
+                       pin=lambda ptr, nbytes: int(rt.cudaHostRegister(ptr, nbytes, 0)) == 0,
+                       unpin=lambda ptr: rt.cudaHostUnregister(ptr))
+
+
+def run_e2e(args, w, spec, host, d, dev, world, local, fn, torch, dist, y_ref=None, r_ref=None, bufs=None):
     norm = "rms" if spec.is_rms else "layer"
     rows = w.rows
     chunk = 4096
-    hy = torch.empty((w.B, w.L, w.D), dtype=torch.bfloat16, pin_memory=True)
-    hr = None if spec.norm_only else torch.empty_like(hy, pin_memory=True)
+    n_out = w.B * w.L * w.D
+    hy = bufs.get("out_y", n_out).view(torch.bfloat16).view(w.B, w.L, w.D)
+    hr = None if spec.norm_only else bufs.get("out_r", n_out).view(torch.bfloat16).view(w.B, w.L, w.D)
     s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
     dy = torch.empty((w.B, w.L, w.D), dtype=torch.bfloat16, device=dev)
     dr = None if spec.norm_only else torch.empty_like(dy)
@@ -639,8 +743,29 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def free_port():
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def launch_ranks(args):
+    """`--gpus N` (N > 1) without a torchrun environment: start the N ranks under
+    torch.distributed.run on this node and return their exit status. Each rank's
+    OpenMP pool gets its share of the host cores."""
+    env = dict(os.environ)
+    env.setdefault("OMP_NUM_THREADS", str(max(1, (os.cpu_count() or 1) // args.gpus)))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={args.gpus}", "--master-addr=127.0.0.1", f"--master-port={free_port()}",
+           os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.run(cmd, env=env).returncode
+
+
 def main():
     args = parse()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(launch_ranks(args))
     if args.impl == "reference":
         run_reference(args)
     else:

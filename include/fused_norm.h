@@ -22,10 +22,15 @@
  * that the affine weight and bias may be fp32 (affine_fp32; the pages' kernel takes fp32
  * affine parameters but casts them to bf16 -- PR 33144, "Known gaps" -- here they are used
  * at full precision).
- * Arithmetic: fp32 for the element-wise work, fp64 for the row statistics; y is the
- * correctly rounded bf16 of the formula evaluated with those statistics, and r the
- * correctly rounded bf16 of the exact residual + gate * x. eps is a runtime value
- * (the pages' kernel hardcodes 1e-6 and ignores the argument; this library does not).
+ * Arithmetic: fp32 for the element-wise work, fp64 for the row statistics. r is the
+ * correctly rounded bf16 of the exact residual + gate * x. y is the bf16 rounding of the
+ * formula evaluated in fp64 with those statistics: the fp32 value is used where its error
+ * bound proves that it rounds the same way, and the other elements (a few in 10^4) are
+ * evaluated in fp64 and rounded once. Against the exact value of the formula y is within
+ * one bf16 ulp (the fp64 evaluation's own last-bit error can only matter for a value
+ * within about 2^-50 of a rounding boundary); on every tested workload it is bit-identical
+ * to the fp64 CPU oracle. eps is a runtime value (the pages' kernel hardcodes 1e-6 and
+ * ignores the argument; this library does not).
  *
  * Operand layouts (PR #33144, "Modifications": a broadcast operand is a dense
  * (1, C) row selected for every token; "Accuracy Tests": per-row scale/shift and the
@@ -48,9 +53,13 @@
  * at once. fused_norm_launch is asynchronous on the given stream.
  *
  * Errors: argument errors are detected on the host, before anything is launched,
- * and leave every output untouched. A failed kernel launch returns FN_ERR_CUDA
- * (the CUDA error is available from fused_norm_last_cuda_error). There is no
- * fallback path of any kind.
+ * and leave every output untouched. FN_ERR_CUDA means the CUDA runtime rejected this
+ * call's kernel launch; the runtime's status for that launch is kept per host thread
+ * (fused_norm_last_cuda_error). The library links its own copy of the CUDA runtime
+ * and reads no error state: an error left pending by an earlier CUDA call, in this
+ * library or in the caller's runtime, is neither reported as this launch's failure
+ * nor cleared. Launches go to the calling thread's current device, which must be the
+ * device that owns the stream and the buffers. There is no fallback path of any kind.
  */
 #ifndef FUSED_NORM_H_
 #define FUSED_NORM_H_
@@ -70,7 +79,7 @@ typedef enum {
   FN_ERR_INVALID_ARG = 1, /* null / inconsistent / negative / overlapping arguments */
   FN_ERR_UNSUPPORTED = 2, /* D not in {5120, 10240} */
   FN_ERR_MISALIGNED = 3,  /* pointer not 16-byte aligned, or stride not a multiple of 8 */
-  FN_ERR_CUDA = 4         /* the kernel launch failed */
+  FN_ERR_CUDA = 4         /* the CUDA runtime rejected this call's kernel launch */
 } fn_status;
 
 typedef struct fused_norm_s* fused_norm_t; /* opaque, host-only */
@@ -162,7 +171,8 @@ fn_status fused_norm_plan(fused_norm_t h, const fn_args* a, int64_t* grid, int* 
 /* Static text for a status code; never NULL. */
 const char* fused_norm_status_string(fn_status s);
 
-/* cudaError_t (as int) of the last FN_ERR_CUDA on this host thread; 0 if none. */
+/* cudaError_t (as int) that the runtime returned for the last launch that ended in
+ * FN_ERR_CUDA on this host thread; 0 if none. Successful launches leave it as it is. */
 int fused_norm_last_cuda_error(void);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */

@@ -15,8 +15,8 @@ fallback path).
 weight and bias are (D,) vectors, bf16 or fp32 (both the same dtype when both are given);
 fp32 values are used at full precision.
 
-Calls are asynchronous on `stream` (default: the current stream of the inputs' device),
-like any PyTorch kernel: when `stream` is not the stream the tensors were produced on, the
+Calls are asynchronous on `stream` (default: the current stream of the inputs' device)
+and run on the inputs' device whichever device is current, like any PyTorch kernel: when `stream` is not the stream the tensors were produced on, the
 caller orders the two streams and keeps the tensors alive (e.g. Tensor.record_stream).
 
 Accepted operand shapes for gate / scale / shift against x of shape (B, L, D):
@@ -130,9 +130,12 @@ def _affine_fp32(weight, bias) -> bool:
 
 
 def _launch(h: int, args: _abi.fn_args, device: torch.device, stream) -> None:
-    if stream is None:
-        stream = torch.cuda.current_stream(device)
-    st = _abi.fused_norm_launch(h, args, int(stream.cuda_stream))
+    # The library launches on the calling thread's current device: make it the tensors'
+    # device for the call (the caller's current device is restored afterwards).
+    with torch.cuda.device(device):
+        if stream is None:
+            stream = torch.cuda.current_stream(device)
+        st = _abi.fused_norm_launch(h, args, int(stream.cuda_stream))
     if st != _abi.FN_OK:
         detail = _abi.fused_norm_status_string(st)
         if st == _abi.FN_ERR_CUDA:

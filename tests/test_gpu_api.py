@@ -1,0 +1,93 @@
+"""GPU checks of the launch contract: which error a launch reports, and which device it
+runs on.
+
+* fused_norm_launch reports the status of its own launch only. An error left pending in
+  the caller's CUDA runtime (here: torch's, by an invalid cudaSetDevice, a host-side
+  argument error that touches no GPU) is neither returned as FN_ERR_CUDA nor cleared.
+* The tensor-level API runs on its inputs' device whichever device is current (needs
+  two GPUs; skipped otherwise).
+"""
+import ctypes
+
+import pytest
+import torch
+
+import rmsnorm_row_b200 as fn
+from rmsnorm_row_b200 import _abi
+
+pytestmark = pytest.mark.gpu
+
+
+def _rand(shape, seed, device, sd=1.0):
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    return (sd * torch.randn(shape, generator=g)).to(torch.bfloat16).to(device)
+
+
+def _caller_runtime():
+    """The CUDA runtime library torch loaded into this process (same instance)."""
+    torch.cuda.init()
+    with open("/proc/self/maps") as f:
+        for line in f:
+            path = line.split()[-1]
+            if "libcudart.so" in path:
+                rt = ctypes.CDLL(path)
+                for name in ("cudaGetLastError", "cudaPeekAtLastError", "cudaSetDevice"):
+                    getattr(rt, name).restype = ctypes.c_int
+                rt.cudaSetDevice.argtypes = [ctypes.c_int]
+                return rt
+    pytest.skip("torch's CUDA runtime is not a separate shared library in this process")
+
+
+def test_launch_neither_reports_nor_clears_a_pending_error():
+    dev = torch.device("cuda:0")
+    B, L, D = 1, 64, 5120
+    x, res = _rand((B, L, D), 1, dev), _rand((B, L, D), 2, dev)
+    gate, scale, shift = (_rand((1, 1, D), s, dev, 0.1) for s in (3, 4, 5))
+    y = torch.empty_like(x)
+    r = torch.empty_like(x)
+    args = fn.build_args(x, res, gate, None, None, scale, shift, y, r)
+    cfg = _abi.fn_config(D=D, is_rms=0, has_gate=1, has_weight=0, has_bias=0, norm_only=0,
+                         affine_fp32=0, eps=1e-6)
+    st, h = _abi.fused_norm_create(cfg)
+    assert st == fn.FN_OK
+    stream = int(torch.cuda.current_stream(dev).cuda_stream)
+    rt = _caller_runtime()
+    try:
+        rt.cudaGetLastError()                       # start clean
+        injected = rt.cudaSetDevice(1 << 20)        # no such device: cudaErrorInvalidDevice
+        assert injected != 0
+        assert rt.cudaPeekAtLastError() == injected
+        # nothing but ctypes calls between the injection and the checks
+        assert _abi.fused_norm_launch(h, args, stream) == fn.FN_OK
+        assert _abi.fused_norm_last_cuda_error() == 0
+        assert rt.cudaPeekAtLastError() == injected  # still pending, for its owner to read
+        assert rt.cudaGetLastError() == injected
+        assert rt.cudaGetLastError() == 0
+        torch.cuda.synchronize(dev)
+        ref_y, ref_r = fn.fused_residual_norm_scale_shift(res, x, gate, None, None, scale, shift,
+                                                          "layer", 1e-6)
+        torch.cuda.synchronize(dev)
+        assert torch.equal(y.view(torch.int16), ref_y.view(torch.int16))
+        assert torch.equal(r.view(torch.int16), ref_r.view(torch.int16))
+    finally:
+        _abi.fused_norm_destroy(h)
+
+
+@pytest.mark.skipif(torch.cuda.device_count() < 2, reason="needs two GPUs")
+def test_api_runs_on_the_inputs_device():
+    d1 = torch.device("cuda:1")
+    B, L, D = 2, 33, 5120
+    x, res = _rand((B, L, D), 11, d1), _rand((B, L, D), 12, d1)
+    gate, scale, shift = _rand((B, L, D), 13, d1, 0.5), _rand((1, D), 14, d1, 0.1), _rand((1, D), 15, d1, 0.1)
+    with torch.cuda.device(d1):
+        want_y, want_r = fn.fused_residual_norm_scale_shift(res, x, gate, None, None, scale, shift)
+        want_n = fn.norm_scale_shift(x, None, None, scale, shift, "rms")
+        torch.cuda.synchronize(d1)
+    torch.cuda.set_device(0)
+    y, r = fn.fused_residual_norm_scale_shift(res, x, gate, None, None, scale, shift)
+    n = fn.norm_scale_shift(x, None, None, scale, shift, "rms")
+    assert torch.cuda.current_device() == 0
+    torch.cuda.synchronize(d1)
+    assert torch.equal(y.view(torch.int16), want_y.view(torch.int16))
+    assert torch.equal(r.view(torch.int16), want_r.view(torch.int16))
+    assert torch.equal(n.view(torch.int16), want_n.view(torch.int16))
