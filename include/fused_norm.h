@@ -137,7 +137,8 @@ fn_status fused_norm_create(fused_norm_t* out, const fn_config* cfg);
  *     use; output rows that overlap one another (y/r stride_l < D when L > 1, or
  *     stride_b < (L-1)*stride_l + D when B > 1); y and r overlapping each other or
  *     any input, except r == residual exactly (same pointer and strides, stride_f 0),
- *     which updates the residual stream in place; sizes whose byte extents overflow.
+ *     which updates the residual stream in place; sizes whose byte extents overflow;
+ *     B * L of 2^31 rows or more (the kernel runs one thread block per row).
  *   FN_ERR_MISALIGNED: a pointer not 16-byte aligned, or a non-zero stride that is
  *     not a multiple of 8 elements (16 bytes).
  *   B * L == 0 is valid (FN_OK) and reads no pointer.

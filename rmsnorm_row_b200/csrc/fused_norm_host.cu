@@ -31,6 +31,7 @@ namespace {
 thread_local int g_last_cuda_error = 0;
 
 constexpr int64_t kMaxExtent = (int64_t)1 << 46;  // elements; keeps byte math in int64
+constexpr int64_t kMaxRows = 0x7FFFFFFFLL;       // B * L: one CTA per row, 32-bit row indices
 
 bool is_flag(int v) { return v == 0 || v == 1; }
 
@@ -79,6 +80,7 @@ fn_status validate(const fused_norm_s* h, const fn_args* a) {
   if (B < 0 || L < 0 || tpf < 0) return FN_ERR_INVALID_ARG;
   if (B == 0 || L == 0) return FN_OK;  // empty problem: nothing is read or written
   if (B > kMaxExtent || L > kMaxExtent || (__int128)B * L * D > kMaxExtent) return FN_ERR_INVALID_ARG;
+  if ((__int128)B * L > (__int128)kMaxRows) return FN_ERR_INVALID_ARG;
   if (tpf > 0 && L % tpf != 0) return FN_ERR_INVALID_ARG;
   const bool frame_axis = tpf > 0;
   const int64_t F = frame_axis ? L / tpf : 1;
@@ -184,9 +186,11 @@ RowParams make_params(const fused_norm_s* h, const fn_args* a) {
   p.shift_sb = a->shift.stride_b; p.shift_sf = a->shift.stride_f; p.shift_sl = a->shift.stride_l;
   p.y_sb = a->y_stride_b; p.y_sl = a->y_stride_l;
   p.r_sb = a->r_stride_b; p.r_sl = a->r_stride_l;
-  p.L = a->L;
-  p.tpf = a->tokens_per_frame;
-  p.rows = a->B * a->L;
+  p.L = (uint32_t)a->L;
+  p.tpf = (uint32_t)a->tokens_per_frame;
+  p.rows = (uint32_t)(a->B * a->L);
+  p.div_L = make_div_u32(p.L);
+  p.div_tpf = make_div_u32(p.tpf > 0 ? p.tpf : 1u);
   p.eps = h->cfg.eps;
   // An operand that changes from token to token (stride_l != 0) is read once per
   // call: stream it. Broadcast, per-batch and per-frame rows are re-read by many
@@ -201,10 +205,7 @@ RowParams make_params(const fused_norm_s* h, const fn_args* a) {
   return p;
 }
 
-int64_t grid_for(int64_t rows) {
-  const int64_t kMaxGrid = 0x7FFFFFFF;  // the kernel loops over rows beyond this
-  return rows < kMaxGrid ? rows : kMaxGrid;
-}
+int64_t grid_for(int64_t rows) { return rows; }  // one CTA per row (B * L <= kMaxRows)
 
 }  // namespace
 

@@ -46,6 +46,30 @@
 
 namespace fused_norm_impl {
 
+// Division of 32-bit values by a divisor fixed for a launch, as a multiply-high and
+// shifts (the branch-free round-up method of Granlund and Montgomery, "Division by
+// invariant integers using multiplication", 1994): for d >= 2, with l = ceil(log2 d)
+// and m = floor(2^32 (2^l - d) / d) + 1, t = mulhi(m, n) gives
+// n / d = (t + ((n - t) >> 1)) >> (l - 1) for every 32-bit n. d == 1 is kept apart.
+struct DivU32 {
+  uint32_t d, m;
+  int shift;  // l - 1
+};
+inline DivU32 make_div_u32(uint32_t d) {
+  DivU32 v{d, 0u, 0};
+  if (d <= 1) return v;
+  int l = 0;
+  while ((uint64_t(1) << l) < d) ++l;
+  v.m = (uint32_t)((((uint64_t(1) << l) - d) << 32) / d + 1);
+  v.shift = l - 1;
+  return v;
+}
+__device__ __forceinline__ uint32_t div_u32(uint32_t n, const DivU32& v) {
+  if (v.d == 1) return n;
+  const uint32_t t = __umulhi(v.m, n);
+  return (t + ((n - t) >> 1)) >> v.shift;
+}
+
 struct RowParams {
   const uint16_t* x;
   const uint16_t* res;
@@ -62,7 +86,8 @@ struct RowParams {
   int64_t scale_sb, scale_sf, scale_sl;
   int64_t shift_sb, shift_sf, shift_sl;
   int64_t y_sb, y_sl, r_sb, r_sl;
-  int64_t L, tpf, rows;
+  uint32_t rows, L, tpf;   // B * L < 2^31 (checked on the host); tpf = 0: no frame axis
+  DivU32 div_L, div_tpf;   // division by L and by tpf (tpf > 0)
   double eps;
   uint32_t stream_mask;  // bit set: operand is per-row (read once) -> streaming load
 };
@@ -438,159 +463,156 @@ fused_norm_rows(const RowParams p) {
   static_assert(T % 32 == 0 && T * 8 * VPT == D, "row must split evenly into warps");
   static_assert(!(NORM_ONLY && HAS_GATE), "norm-only has no gate");
 
-  __shared__ double2 part[2][W];
+  __shared__ double2 part[W];
   __shared__ double centred[W];
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
-  int parity = 0;
 
-  for (int64_t row = blockIdx.x; row < p.rows; row += gridDim.x, parity ^= 1) {
-    const int64_t b = row / p.L;
-    const int64_t l = row - b * p.L;
-    const int64_t f = p.tpf > 0 ? l / p.tpf : 0;
+  // One row per CTA: the grid is B * L (< 2^31, checked on the host).
+  const uint32_t row = blockIdx.x;
+  const uint32_t b = div_u32(row, p.div_L);
+  const uint32_t l = row - b * p.L;
+  const uint32_t f = p.tpf > 0 ? div_u32(l, p.div_tpf) : 0u;
 
-    const uint16_t* xr = p.x + (b * p.x_sb + f * p.x_sf + l * p.x_sl);
-    const uint16_t* sr = p.scale + (b * p.scale_sb + f * p.scale_sf + l * p.scale_sl);
-    const uint16_t* tr = p.shift + (b * p.shift_sb + f * p.shift_sf + l * p.shift_sl);
+  const uint16_t* xr = p.x + (b * p.x_sb + f * p.x_sf + l * p.x_sl);
+  const uint16_t* sr = p.scale + (b * p.scale_sb + f * p.scale_sf + l * p.scale_sl);
+  const uint16_t* tr = p.shift + (b * p.shift_sb + f * p.shift_sf + l * p.shift_sl);
 
-    // ---- loads: x, residual and gate are requested together. scale and shift are
-    // requested with them or right after the r stores (FN_EARLY_MODULATION_LOADS);
-    // a load written after a store waits for the store's issue, since the compiler
-    // cannot rule out aliasing.
-    uint4 xv[VPT], rv[VPT], gv[VPT], sv[VPT], tv[VPT];
+  // ---- loads: x, residual and gate are requested together. scale and shift are
+  // requested with them or right after the r stores (FN_EARLY_MODULATION_LOADS);
+  // a load written after a store waits for the store's issue, since the compiler
+  // cannot rule out aliasing.
+  uint4 xv[VPT], rv[VPT], gv[VPT], sv[VPT], tv[VPT];
 #pragma unroll
+  for (int k = 0; k < VPT; ++k) xv[k] = load_vec(xr, tid + k * T, p.stream_mask & kX);
+  if (!NORM_ONLY) {
+    const uint16_t* rr = p.res + (b * p.res_sb + f * p.res_sf + l * p.res_sl);
 #pragma unroll
-    for (int k = 0; k < VPT; ++k) xv[k] = load_vec(xr, tid + k * T, p.stream_mask & kX);
-    if (!NORM_ONLY) {
-      const uint16_t* rr = p.res + (b * p.res_sb + f * p.res_sf + l * p.res_sl);
+    for (int k = 0; k < VPT; ++k) rv[k] = load_vec(rr, tid + k * T, p.stream_mask & kRes);
+  }
+  if (HAS_GATE) {
+    const uint16_t* gr = p.gate + (b * p.gate_sb + f * p.gate_sf + l * p.gate_sl);
 #pragma unroll
-      for (int k = 0; k < VPT; ++k) rv[k] = load_vec(rr, tid + k * T, p.stream_mask & kRes);
-    }
-    if (HAS_GATE) {
-      const uint16_t* gr = p.gate + (b * p.gate_sb + f * p.gate_sf + l * p.gate_sl);
-#pragma unroll
-      for (int k = 0; k < VPT; ++k) gv[k] = load_vec(gr, tid + k * T, p.stream_mask & kGate);
-    }
-    if (FN_EARLY_MODULATION_LOADS && !CACHED_MOD) {
-#pragma unroll
-      for (int k = 0; k < VPT; ++k) {
-        sv[k] = load_vec(sr, tid + k * T, p.stream_mask & kScale);
-        tv[k] = load_vec(tr, tid + k * T, p.stream_mask & kShift);
-      }
-    }
-
-    // ---- step 1: r = residual + gate * x, rounded to bf16, stored -------------
-    uint4 v[VPT];  // the row (r, or x when norm-only), packed bf16 pairs
-    if (NORM_ONLY) {
-#pragma unroll
-      for (int k = 0; k < VPT; ++k) v[k] = xv[k];
-    } else {
-      uint4* ro = reinterpret_cast<uint4*>(p.r + (b * p.r_sb + l * p.r_sl));
-#pragma unroll
-      for (int k = 0; k < VPT; ++k) {
-        v[k] = residual_vec<HAS_GATE>(rv[k], xv[k], HAS_GATE ? gv[k] : rv[k]);
-        __stcs(ro + tid + k * T, v[k]);
-      }
-    }
-
-    if (!FN_EARLY_MODULATION_LOADS && !CACHED_MOD) {
-#pragma unroll
-      for (int k = 0; k < VPT; ++k) {
-        sv[k] = load_vec(sr, tid + k * T, p.stream_mask & kScale);
-        tv[k] = load_vec(tr, tid + k * T, p.stream_mask & kShift);
-      }
-    }
-
-    // ---- step 2: row statistics in fp64 ------------------------------------
-    // Four independent accumulation chains per thread (one per word of a vector),
-    // combined in a fixed order: short dependency chains, reproducible sums.
-    double a1[4] = {0.0, 0.0, 0.0, 0.0}, a2[4] = {0.0, 0.0, 0.0, 0.0};
-#pragma unroll
-    for (int k = 0; k < VPT; ++k)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const double a = bf16_f64<0>(word(v[k], i)), c = bf16_f64<1>(word(v[k], i));
-        if (!IS_RMS) a1[i] += a + c;                 // a + c exact: two bf16 values
-        if (NORM_ONLY)
-          a2[i] = fma(c, c, fma(a, a, a2[i]));       // squares of bf16 values: exact
-        else
-          a2[i] += fma(a, a, c * c);                 // c * c exact (16-bit significand)
-      }
-    double s1 = (a1[0] + a1[1]) + (a1[2] + a1[3]);
-    double s2 = (a2[0] + a2[1]) + (a2[2] + a2[3]);
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-      if (!IS_RMS) s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, o);
-      s2 += __shfl_xor_sync(0xFFFFFFFFu, s2, o);
-    }
-    if (lane == 0) part[parity][warp] = make_double2(s1, s2);
-    __syncthreads();
-    double t1 = part[parity][0].x, t2 = part[parity][0].y;
-#pragma unroll
-    for (int w = 1; w < W; ++w) {
-      t1 += part[parity][w].x;
-      t2 += part[parity][w].y;
-    }
-    // Correctly rounded divisions by D (not products with 1/D): the mean is then the
-    // rounded quotient of the exact sum, as defined, and a row whose mean dwarfs its
-    // spread does not turn a last-bit difference of the mean into a different output.
-    RowStats st;
-    if (IS_RMS) {
-      st.mu = 0.0;
-      st.rho = rsqrt(div_by_row_length<D>(t2) + p.eps);
-    } else {
-      const double mu = div_by_row_length<D>(t1);
-      double var = fmax(div_by_row_length<D>(t2) - mu * mu, 0.0);
-      if (mu * mu > 1048576.0 * var && var > 0.0) {
-        // The mean dwarfs the spread: take the variance around the mean instead
-        // (uniform branch: every thread of the CTA has the same statistics). The row
-        // is read back from memory (this thread's own r stores, or x) in a rolled
-        // loop: unrolled over the register copy, this rare pass would set the
-        // kernel's register allocation and force spills on the common path.
-        const uint4* rowv = NORM_ONLY ? reinterpret_cast<const uint4*>(xr)
-                                      : reinterpret_cast<const uint4*>(p.r + (b * p.r_sb + l * p.r_sl));
-        double c2 = 0.0;
-#pragma unroll 1
-        for (int k = 0; k < VPT; ++k) {
-          const uint4 vk = __ldcg(rowv + tid + k * T);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const double a = bf16_f64<0>(word(vk, i)) - mu, c = bf16_f64<1>(word(vk, i)) - mu;
-            c2 = fma(a, a, c2);
-            c2 = fma(c, c, c2);
-          }
-        }
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) c2 += __shfl_xor_sync(0xFFFFFFFFu, c2, o);
-        if (lane == 0) centred[warp] = c2;
-        __syncthreads();
-        double tc = centred[0];
-#pragma unroll
-        for (int w = 1; w < W; ++w) tc += centred[w];
-        var = div_by_row_length<D>(tc);
-        __syncthreads();  // centred[] is reused by the next such row
-      }
-      st.mu = mu;
-      st.rho = rsqrt(var + p.eps);
-    }
-    st.neg_mu32 = -(float)st.mu;
-    st.rho32 = (float)st.rho;
-    st.kappa = fabsf(st.neg_mu32) * st.rho32;
-
-    // ---- step 3: normalise, affine, modulate, store y ------------------------
-    uint4* yo = reinterpret_cast<uint4*>(p.y + (b * p.y_sb + l * p.y_sl));
+    for (int k = 0; k < VPT; ++k) gv[k] = load_vec(gr, tid + k * T, p.stream_mask & kGate);
+  }
+  if (FN_EARLY_MODULATION_LOADS && !CACHED_MOD) {
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
-      const int j = tid + k * T;
-      if (CACHED_MOD) {  // broadcast / per-frame rows: L1 hits, fetched as they are used
-        sv[k] = __ldg(reinterpret_cast<const uint4*>(sr) + j);
-        tv[k] = __ldg(reinterpret_cast<const uint4*>(tr) + j);
-      }
-      using Affine = typename std::conditional<AFFINE_F32, AffineF32, AffineBF16>::type;
-      const Affine wf = HAS_WEIGHT ? Affine::load(p.weight, j) : Affine::fill(1.0f);
-      const Affine bf = HAS_BIAS ? Affine::load(p.bias, j) : Affine::fill(0.0f);
-      __stcs(yo + j, output_vec<RowShape<D>::kPaired, HAS_WEIGHT, HAS_BIAS>(v[k], sv[k], tv[k], wf, bf, st));
+      sv[k] = load_vec(sr, tid + k * T, p.stream_mask & kScale);
+      tv[k] = load_vec(tr, tid + k * T, p.stream_mask & kShift);
     }
+  }
+
+  // ---- step 1: r = residual + gate * x, rounded to bf16, stored -------------
+  uint4 v[VPT];  // the row (r, or x when norm-only), packed bf16 pairs
+  if (NORM_ONLY) {
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) v[k] = xv[k];
+  } else {
+    uint4* ro = reinterpret_cast<uint4*>(p.r + (b * p.r_sb + l * p.r_sl));
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      v[k] = residual_vec<HAS_GATE>(rv[k], xv[k], HAS_GATE ? gv[k] : rv[k]);
+      __stcs(ro + tid + k * T, v[k]);
+    }
+  }
+
+  if (!FN_EARLY_MODULATION_LOADS && !CACHED_MOD) {
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      sv[k] = load_vec(sr, tid + k * T, p.stream_mask & kScale);
+      tv[k] = load_vec(tr, tid + k * T, p.stream_mask & kShift);
+    }
+  }
+
+  // ---- step 2: row statistics in fp64 ------------------------------------
+  // Four independent accumulation chains per thread (one per word of a vector),
+  // combined in a fixed order: short dependency chains, reproducible sums.
+  double a1[4] = {0.0, 0.0, 0.0, 0.0}, a2[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+  for (int k = 0; k < VPT; ++k)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const double a = bf16_f64<0>(word(v[k], i)), c = bf16_f64<1>(word(v[k], i));
+      if (!IS_RMS) a1[i] += a + c;                 // a + c exact: two bf16 values
+      if (NORM_ONLY)
+        a2[i] = fma(c, c, fma(a, a, a2[i]));       // squares of bf16 values: exact
+      else
+        a2[i] += fma(a, a, c * c);                 // c * c exact (16-bit significand)
+    }
+  double s1 = (a1[0] + a1[1]) + (a1[2] + a1[3]);
+  double s2 = (a2[0] + a2[1]) + (a2[2] + a2[3]);
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    if (!IS_RMS) s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, o);
+    s2 += __shfl_xor_sync(0xFFFFFFFFu, s2, o);
+  }
+  if (lane == 0) part[warp] = make_double2(s1, s2);
+  __syncthreads();
+  double t1 = part[0].x, t2 = part[0].y;
+#pragma unroll
+  for (int w = 1; w < W; ++w) {
+    t1 += part[w].x;
+    t2 += part[w].y;
+  }
+  // Correctly rounded divisions by D (not products with 1/D): the mean is then the
+  // rounded quotient of the exact sum, as defined, and a row whose mean dwarfs its
+  // spread does not turn a last-bit difference of the mean into a different output.
+  RowStats st;
+  if (IS_RMS) {
+    st.mu = 0.0;
+    st.rho = rsqrt(div_by_row_length<D>(t2) + p.eps);
+  } else {
+    const double mu = div_by_row_length<D>(t1);
+    double var = fmax(div_by_row_length<D>(t2) - mu * mu, 0.0);
+    if (mu * mu > 1048576.0 * var && var > 0.0) {
+      // The mean dwarfs the spread: take the variance around the mean instead
+      // (uniform branch: every thread of the CTA has the same statistics). The row
+      // is read back from memory (this thread's own r stores, or x) in a rolled
+      // loop: unrolled over the register copy, this rare pass would set the
+      // kernel's register allocation and force spills on the common path.
+      const uint4* rowv = NORM_ONLY ? reinterpret_cast<const uint4*>(xr)
+                                    : reinterpret_cast<const uint4*>(p.r + (b * p.r_sb + l * p.r_sl));
+      double c2 = 0.0;
+#pragma unroll 1
+      for (int k = 0; k < VPT; ++k) {
+        const uint4 vk = __ldcg(rowv + tid + k * T);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const double a = bf16_f64<0>(word(vk, i)) - mu, c = bf16_f64<1>(word(vk, i)) - mu;
+          c2 = fma(a, a, c2);
+          c2 = fma(c, c, c2);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) c2 += __shfl_xor_sync(0xFFFFFFFFu, c2, o);
+      if (lane == 0) centred[warp] = c2;
+      __syncthreads();
+      double tc = centred[0];
+#pragma unroll
+      for (int w = 1; w < W; ++w) tc += centred[w];
+      var = div_by_row_length<D>(tc);
+    }
+    st.mu = mu;
+    st.rho = rsqrt(var + p.eps);
+  }
+  st.neg_mu32 = -(float)st.mu;
+  st.rho32 = (float)st.rho;
+  st.kappa = fabsf(st.neg_mu32) * st.rho32;
+
+  // ---- step 3: normalise, affine, modulate, store y ------------------------
+  uint4* yo = reinterpret_cast<uint4*>(p.y + (b * p.y_sb + l * p.y_sl));
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) {
+    const int j = tid + k * T;
+    if (CACHED_MOD) {  // broadcast / per-frame rows: L1 hits, fetched as they are used
+      sv[k] = __ldg(reinterpret_cast<const uint4*>(sr) + j);
+      tv[k] = __ldg(reinterpret_cast<const uint4*>(tr) + j);
+    }
+    using Affine = typename std::conditional<AFFINE_F32, AffineF32, AffineBF16>::type;
+    const Affine wf = HAS_WEIGHT ? Affine::load(p.weight, j) : Affine::fill(1.0f);
+    const Affine bf = HAS_BIAS ? Affine::load(p.bias, j) : Affine::fill(0.0f);
+    __stcs(yo + j, output_vec<RowShape<D>::kPaired, HAS_WEIGHT, HAS_BIAS>(v[k], sv[k], tv[k], wf, bf, st));
   }
 }
 

@@ -235,6 +235,15 @@ def test_extent_overflow_is_rejected():
     assert fn.fused_norm_validate(h, a) == INV
 
 
+def test_row_count_limit():
+    # one CTA per row with 32-bit row indices: B * L must stay below 2^31
+    h = make()
+    assert fn.fused_norm_validate(h, valid_args(B=1, L=(1 << 31) - 1)) == OK
+    assert fn.fused_norm_validate(h, valid_args(B=1, L=1 << 31)) == INV
+    assert fn.fused_norm_validate(h, valid_args(B=2, L=1 << 30)) == INV
+    assert fn.fused_norm_validate(h, valid_args(B=3, L=(1 << 31) // 3)) == OK
+
+
 def test_null_handle_and_args():
     assert fn.load().fused_norm_validate(None, None) == INV
     h = make()
