@@ -424,9 +424,7 @@ template <int D> struct RowShape;
 #endif
 // Norm-only with broadcast / per-frame scale and shift reads one tensor and writes one
 // per row, so its per-element arithmetic, not HBM, sets its pace: those instances run
-// 7 CTAs per SM (72 registers), one more than the other broadcast instances, and sum
-// squares with two fused multiply-adds per pair (one instruction fewer; where the
-// other instances' register budgets leave no room for it, they keep the product form).
+// 7 CTAs per SM (68 registers), one more than the other broadcast instances.
 #ifndef FN_MINB_NSS_5120
 #define FN_MINB_NSS_5120 7
 #endif
@@ -446,7 +444,11 @@ template <> struct RowShape<10240> {
   static constexpr bool kPaired = FN_PAIRED_10240 != 0;
 };
 
-// CTAs per SM an instance's register budget is sized for.
+// CTAs per SM an instance's register budget is sized for. The figure is per D and
+// operand placement, the same for every specialisation: instances that carry more live
+// values (fp32 affine, bias, RMSNorm with weight at D = 10240) spill a few registers to
+// L1 at these counts, and measured faster so than with one CTA fewer (D = 10240,
+// broadcast modulation: 1.15 ms with 3 CTAs per SM and spills, 1.30 ms with 2 and none).
 template <int D, bool NORM_ONLY, bool CACHED_MOD>
 constexpr int min_blocks() {
   return (NORM_ONLY && CACHED_MOD) ? RowShape<D>::kMinBlocksNss
@@ -535,10 +537,7 @@ fused_norm_rows(const RowParams p) {
     for (int i = 0; i < 4; ++i) {
       const double a = bf16_f64<0>(word(v[k], i)), c = bf16_f64<1>(word(v[k], i));
       if (!IS_RMS) a1[i] += a + c;                 // a + c exact: two bf16 values
-      if (NORM_ONLY)
-        a2[i] = fma(c, c, fma(a, a, a2[i]));       // squares of bf16 values: exact
-      else
-        a2[i] += fma(a, a, c * c);                 // c * c exact (16-bit significand)
+      a2[i] = fma(c, c, fma(a, a, a2[i]));         // squares of bf16 values: exact
     }
   double s1 = (a1[0] + a1[1]) + (a1[2] + a1[3]);
   double s2 = (a2[0] + a2[1]) + (a2[2] + a2[3]);
