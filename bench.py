@@ -68,6 +68,9 @@ def parse():
     p.add_argument("--flush-l2", action="store_true",
                    help="write a 512 MB buffer before every timed launch and time each launch "
                         "alone (for the small shapes, whose inputs otherwise stay in L2)")
+    p.add_argument("--affine-fp32", action="store_true",
+                   help="weight and bias as fp32 (used at full precision), as the pages' "
+                        "microbenchmark passes them")
     p.add_argument("--graph", action="store_true",
                    help="replay the timed launches from one CUDA graph (removes host launch "
                         "overhead; for the launch-bound small shapes)")
@@ -94,11 +97,13 @@ def workload(args):
     return w
 
 
-def config_dict(w, spec, n):
+def config_dict(w, spec, n, affine_fp32=False):
     lay = {op: w.layout(op) for op in ("gate", "scale", "shift")}
     return {"workload": w.name, "spec": spec.name, "B": w.B, "L": w.L, "D": w.D, "frames": w.F or None,
             "norm": "rms" if spec.is_rms else "layer", "has_gate": spec.has_gate,
-            "has_weight": spec.has_weight, "layouts": lay, "eps": w.eps,
+            "has_weight": spec.has_weight, "has_bias": spec.has_bias,
+            "affine_dtype": ("fp32" if affine_fp32 else "bf16") if (spec.has_weight or spec.has_bias) else None,
+            "layouts": lay, "eps": w.eps,
             "parallelism": f"rows per rank, {n} independent problem(s)" if n > 1 else "single GPU",
             "l2": "inputs larger than L2 (no flush needed)" if w.algorithmic_bytes(spec) > 4 * 126e6
                   else "L2-resident (small case)"}
@@ -262,6 +267,11 @@ def run_ours(args):
                 or name == "bias" and not spec.has_bias \
                 or name in ("residual", "gate") and spec.norm_only:
             continue
+        if name in ("weight", "bias") and args.affine_fp32:
+            t = bufs.get(f"in_{name}", 2 * w.D,
+                         lambda a, name=name: a.view(np.float32).__setitem__(slice(None), w.generate_f32(name)))
+            host[name] = t.view(torch.float32).view(w.D)
+            continue
         n = 1 if name in ("weight", "bias") else w.stored_rows(name)
         t = bufs.get(f"in_{name}", n * w.D, lambda a, name=name: w.generate(name, out=a.reshape(-1, w.D)))
         host[name] = t.view(torch.bfloat16).view(synth.device.operand_view_shape(w, name))
@@ -275,8 +285,11 @@ def run_ours(args):
     # ~15 us of host time and dominates the launch-bound small shapes).
     args_c = fn.build_args(d["x"], d.get("residual"), d.get("gate"), d.get("weight"), d.get("bias"),
                            d["scale"], d["shift"], y, r)
+    affine_fp32 = bool(args.affine_fp32 and (spec.has_weight or spec.has_bias))
+    if affine_fp32:   # fp32 weight / bias: 4 bytes per channel instead of 2
+        bytes_step += 2 * w.D * (int(spec.has_weight) + int(spec.has_bias))
     handle = fn.api._handle(w.D, spec.is_rms, spec.has_gate, spec.has_weight, spec.has_bias,
-                            spec.norm_only, w.eps, False)
+                            spec.norm_only, w.eps, affine_fp32)
 
     def step():
         st = fn.fused_norm_launch(handle, args_c, int(stream.cuda_stream))
@@ -390,7 +403,7 @@ def run_ours(args):
             "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded normal draws, WAN2.2 shapes; no model weights)",
-            "config": dict(config_dict(w, spec, world), launch="cuda_graph" if graph is not None else "stream",
+            "config": dict(config_dict(w, spec, world, affine_fp32), launch="cuda_graph" if graph is not None else "stream",
                            **({"l2": "flushed before every timed launch (512 MB write, outside the "
                                      "per-launch events)"} if scratch is not None else {})),
             "rows_per_s": round(world * w.rows / (ms_step * 1e-3), 1),
@@ -646,7 +659,8 @@ def cpu_baseline(w, spec, host, seconds):
     import oracle
     if w.B != 1 or w.F:
         return None
-    host_np = {k: v.view(torch_int16()).numpy().view(np.uint16).reshape(-1, w.D) for k, v in host.items()}
+    host_np = {k: (v.numpy() if v.dtype == torch_float32() else
+                   v.view(torch_int16()).numpy().view(np.uint16).reshape(-1, w.D)) for k, v in host.items()}
     per_row_bytes = w.algorithmic_bytes(spec) / w.rows
     done, t0, chunk = 0, time.time(), 1024
     while time.time() - t0 < seconds and done < w.rows:
@@ -688,6 +702,11 @@ def torch_int16():
     return torch.int16
 
 
+def torch_float32():
+    import torch
+    return torch.float32
+
+
 def run_reference(args):
     """The fp64 oracle on the host cores, K timed steps of a bounded row sample."""
     import oracle
@@ -711,6 +730,9 @@ def run_reference(args):
     def gen(rows):
         out = {}
         for name in names:
+            if name in ("weight", "bias") and args.affine_fp32:
+                out[name] = w.generate_f32(name)
+                continue
             per_token = name in ("x", "residual") or (name not in ("weight", "bias") and w.layout(name) == "row")
             out[name] = w.generate(name, np.arange(rows if per_token else 1, dtype=np.int64))
         return out
@@ -734,7 +756,7 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded normal draws, WAN2.2 shapes)", "impl": "reference",
-            "config": config_dict(w, spec, 1),
+            "config": config_dict(w, spec, 1, bool(args.affine_fp32 and (spec.has_weight or spec.has_bias))),
             "rows_per_s": round(rows / (ms * 1e-3), 1),
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": oracle.num_threads(),
                              "kind": "oracle", "sample": f"first {rows} of {w.rows} rows per step"},

@@ -64,9 +64,13 @@ inline DivU32 make_div_u32(uint32_t d) {
   v.shift = l - 1;
   return v;
 }
-__device__ __forceinline__ uint32_t div_u32(uint32_t n, const DivU32& v) {
+__host__ __device__ __forceinline__ uint32_t div_u32(uint32_t n, const DivU32& v) {
   if (v.d == 1) return n;
+#ifdef __CUDA_ARCH__
   const uint32_t t = __umulhi(v.m, n);
+#else
+  const uint32_t t = (uint32_t)(((uint64_t)v.m * n) >> 32);
+#endif
   return (t + ((n - t) >> 1)) >> v.shift;
 }
 
