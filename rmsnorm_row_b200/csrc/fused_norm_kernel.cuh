@@ -449,20 +449,23 @@ template <> struct RowShape<10240> {
 };
 
 // CTAs per SM an instance's register budget is sized for. The figure is per D and
-// operand placement, the same for every specialisation: instances that carry more live
-// values (fp32 affine, bias, RMSNorm with weight at D = 10240) spill a few registers to
-// L1 at these counts, and measured faster so than with one CTA fewer (D = 10240,
-// broadcast modulation: 1.15 ms with 3 CTAs per SM and spills, 1.30 ms with 2 and none).
-template <int D, bool NORM_ONLY, bool CACHED_MOD>
+// operand placement: instances that carry more live values (fp32 affine, bias, RMSNorm
+// with weight at D = 10240) spill a few registers to L1 at these counts, and most measured
+// faster so than with one CTA fewer (D = 10240, broadcast modulation: 1.15 ms with 3 CTAs
+// per SM and spills, 1.30 ms with 2 and none). The exception is an fp32 bias with cached
+// modulation, whose 16 fp32 affine values per vector spill ~90 bytes at 6 CTAs: one CTA
+// fewer is 4% faster there (the pages' broadcast shape with fp32 w and b), while fp32
+// weight alone is 2% slower with one CTA fewer.
+template <int D, bool NORM_ONLY, bool CACHED_MOD, bool AFFINE_F32, bool HAS_BIAS>
 constexpr int min_blocks() {
   return (NORM_ONLY && CACHED_MOD) ? RowShape<D>::kMinBlocksNss
-         : CACHED_MOD              ? RowShape<D>::kMinBlocksCachedMod
-                                   : RowShape<D>::kMinBlocks;
+         : CACHED_MOD ? RowShape<D>::kMinBlocksCachedMod - ((AFFINE_F32 && HAS_BIAS && D == 5120) ? 1 : 0)
+                      : RowShape<D>::kMinBlocks;
 }
 
 template <int D, int VPT, bool IS_RMS, bool NORM_ONLY, bool HAS_GATE, bool HAS_WEIGHT, bool HAS_BIAS,
           bool AFFINE_F32, bool CACHED_MOD>
-__global__ void __launch_bounds__(D / (8 * VPT), (min_blocks<D, NORM_ONLY, CACHED_MOD>()))
+__global__ void __launch_bounds__(D / (8 * VPT), (min_blocks<D, NORM_ONLY, CACHED_MOD, AFFINE_F32, HAS_BIAS>()))
 fused_norm_rows(const RowParams p) {
   constexpr int T = D / (8 * VPT);
   constexpr int W = T / 32;
