@@ -146,18 +146,27 @@ def test_microbench_bcast_B1_L176400_full(spec):
 # ---- fp32 affine parameters ----------------------------------------------------------
 
 @pytest.mark.parametrize("D", [5120, 10240])
+@pytest.mark.parametrize("layouts", [("bcast", "row", "row"), ("bcast", "bcast", "bcast"),
+                                     ("frame", "frame", "frame")], ids=lambda l: "-".join(l))
 @pytest.mark.parametrize("spec", [synth.Spec(False, True, True, has_bias=True),
+                                  synth.Spec(True, True, True, has_bias=True),
                                   synth.Spec(True, False, True),
+                                  synth.Spec(False, True, True),
                                   synth.Spec(False, False, False, has_bias=True),
                                   synth.Spec(True, False, True, has_bias=True, norm_only=True)],
                          ids=lambda s: s.name)
-def test_fp32_affine(D, spec):
+def test_fp32_affine(D, layouts, spec):
     # weight and bias as fp32 (the same draws as the bf16 ones, kept at 24 bits), used at
-    # full precision on both sides
-    import oracle
+    # full precision on both sides. Per-row scale/shift run the instances that load them
+    # with x; broadcast and per-frame ones the instances that fetch them from L1 (with a
+    # CTA count of their own for an fp32 bias). L = 531 = 9 frames of 59 tokens.
     from parity import oracle_rows
     base = synth.W3 if D == 5120 else synth.W3B
-    w = synth.scaled(base, 613)
+    w = synth.scaled(base, 531)
+    w = synth.dataclasses.replace(w, F=9 if "frame" in layouts else 0,
+                                  layouts=(("gate", layouts[0]), ("scale", layouts[1]),
+                                           ("shift", layouts[2])),
+                                  name=f"{w.name}_{'-'.join(layouts)}")
     host = host_inputs(w)
     dev = upload_host(w, host, DEV)
     w32 = torch.from_numpy(w.generate_f32("weight")).to(DEV) if spec.has_weight else None
