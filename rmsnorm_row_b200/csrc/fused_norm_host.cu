@@ -245,8 +245,9 @@ fn_status fused_norm_create(fused_norm_t* out, const fn_config* cfg) {
   h->launch = fn;
   h->launch_cached_mod = fn_cm;
   h->threads = c.D / (8 * (c.D == 5120 ? RowShape<5120>::VPT : RowShape<10240>::VPT));
-  h->threads_cached_mod =
-      c.D / (8 * (c.D == 5120 ? RowShape<5120>::kVptCachedMod : RowShape<10240>::kVptCachedMod));
+  const int vpt_cm = c.norm_only ? (c.D == 5120 ? RowShape<5120>::kVptNss : RowShape<10240>::kVptNss)
+                                 : (c.D == 5120 ? RowShape<5120>::kVptCachedMod : RowShape<10240>::kVptCachedMod);
+  h->threads_cached_mod = c.D / (8 * vpt_cm);
   *out = h;
   return FN_OK;
 }

@@ -432,19 +432,28 @@ template <int D> struct RowShape;
 #ifndef FN_MINB_NSS_5120
 #define FN_MINB_NSS_5120 7
 #endif
+#ifndef FN_VPT_NSS_5120
+#define FN_VPT_NSS_5120 FN_VPT_5120
+#endif
+// At D = 10240 they take 256 threads x 5 vectors at 4 CTAs per SM instead of 320 x 4 at
+// 3: measured 0.79 -> 0.69 ms on a broadcast norm-only shape (L = 90000). The fused
+// instances with cached modulation keep 320 x 4 (256 x 5 is mixed there: -2% to +3%).
 #ifndef FN_MINB_NSS_10240
-#define FN_MINB_NSS_10240 FN_MINB_CM_10240
+#define FN_MINB_NSS_10240 4
+#endif
+#ifndef FN_VPT_NSS_10240
+#define FN_VPT_NSS_10240 5
 #endif
 template <> struct RowShape<5120> {
   static constexpr int VPT = FN_VPT_5120, kMinBlocks = FN_MINB_5120;
   static constexpr int kMinBlocksCachedMod = FN_MINB_CM_5120, kVptCachedMod = FN_VPT_CM_5120;
-  static constexpr int kMinBlocksNss = FN_MINB_NSS_5120;
+  static constexpr int kMinBlocksNss = FN_MINB_NSS_5120, kVptNss = FN_VPT_NSS_5120;
   static constexpr bool kPaired = FN_PAIRED_5120 != 0;
 };
 template <> struct RowShape<10240> {
   static constexpr int VPT = FN_VPT_10240, kMinBlocks = FN_MINB_10240;
   static constexpr int kMinBlocksCachedMod = FN_MINB_CM_10240, kVptCachedMod = FN_VPT_CM_10240;
-  static constexpr int kMinBlocksNss = FN_MINB_NSS_10240;
+  static constexpr int kMinBlocksNss = FN_MINB_NSS_10240, kVptNss = FN_VPT_NSS_10240;
   static constexpr bool kPaired = FN_PAIRED_10240 != 0;
 };
 
@@ -639,7 +648,7 @@ cudaError_t launch_rows(const RowParams& p, int64_t grid, cudaStream_t stream) {
 // Launcher for one (norm_only, gate, modulation caching) group: the affine combinations.
 template <int D, bool RMS, bool NO, bool G, bool CM>
 LaunchFn pick_affine(bool w, bool b, bool f32) {
-  constexpr int V = CM ? RowShape<D>::kVptCachedMod : RowShape<D>::VPT;
+  constexpr int V = (NO && CM) ? RowShape<D>::kVptNss : CM ? RowShape<D>::kVptCachedMod : RowShape<D>::VPT;
   if (!w && !b) return &launch_rows<D, V, RMS, NO, G, false, false, false, CM>;
   if (f32) {
     if (w && b) return &launch_rows<D, V, RMS, NO, G, true, true, true, CM>;
