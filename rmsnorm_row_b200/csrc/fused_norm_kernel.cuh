@@ -420,11 +420,16 @@ template <int D> struct RowShape;
 #ifndef FN_PAIRED_10240
 #define FN_PAIRED_10240 1
 #endif
-// 1: scale/shift loads are issued with x and residual, before the r stores;
-// 0: after them, where the statistics' reduction and barrier hide their latency
-// (fewer live registers; measured faster on B200 for the WAN2.2 shape).
-#ifndef FN_EARLY_MODULATION_LOADS
-#define FN_EARLY_MODULATION_LOADS 0
+// 1: per-row scale/shift loads are issued with x and residual, before the r stores;
+// 0: after them, where the statistics' reduction and barrier hide their latency (fewer
+// live registers). Measured on B200: 0 is faster at D = 5120 (WAN2.2 shape), 1 at
+// D = 10240, whose two CTAs per SM leave registers to spare (0.4-2% on all its per-row
+// specialisations).
+#ifndef FN_EARLY_MODULATION_LOADS_5120
+#define FN_EARLY_MODULATION_LOADS_5120 0
+#endif
+#ifndef FN_EARLY_MODULATION_LOADS_10240
+#define FN_EARLY_MODULATION_LOADS_10240 1
 #endif
 // Norm-only with broadcast / per-frame scale and shift reads one tensor and writes one
 // per row, so its per-element arithmetic, not HBM, sets its pace: those instances run
@@ -450,12 +455,14 @@ template <> struct RowShape<5120> {
   static constexpr int kMinBlocksCachedMod = FN_MINB_CM_5120, kVptCachedMod = FN_VPT_CM_5120;
   static constexpr int kMinBlocksNss = FN_MINB_NSS_5120, kVptNss = FN_VPT_NSS_5120;
   static constexpr bool kPaired = FN_PAIRED_5120 != 0;
+  static constexpr bool kEarlyModLoads = FN_EARLY_MODULATION_LOADS_5120 != 0;
 };
 template <> struct RowShape<10240> {
   static constexpr int VPT = FN_VPT_10240, kMinBlocks = FN_MINB_10240;
   static constexpr int kMinBlocksCachedMod = FN_MINB_CM_10240, kVptCachedMod = FN_VPT_CM_10240;
   static constexpr int kMinBlocksNss = FN_MINB_NSS_10240, kVptNss = FN_VPT_NSS_10240;
   static constexpr bool kPaired = FN_PAIRED_10240 != 0;
+  static constexpr bool kEarlyModLoads = FN_EARLY_MODULATION_LOADS_10240 != 0;
 };
 
 // CTAs per SM an instance's register budget is sized for. The figure is per D and
@@ -498,7 +505,7 @@ fused_norm_rows(const RowParams p) {
   const uint16_t* tr = p.shift + (b * p.shift_sb + f * p.shift_sf + l * p.shift_sl);
 
   // ---- loads: x, residual and gate are requested together. scale and shift are
-  // requested with them or right after the r stores (FN_EARLY_MODULATION_LOADS);
+  // requested with them or right after the r stores (RowShape<D>::kEarlyModLoads);
   // a load written after a store waits for the store's issue, since the compiler
   // cannot rule out aliasing.
   uint4 xv[VPT], rv[VPT], gv[VPT], sv[VPT], tv[VPT];
@@ -514,7 +521,7 @@ fused_norm_rows(const RowParams p) {
 #pragma unroll
     for (int k = 0; k < VPT; ++k) gv[k] = load_vec(gr, tid + k * T, p.stream_mask & kGate);
   }
-  if (FN_EARLY_MODULATION_LOADS && !CACHED_MOD) {
+  if (RowShape<D>::kEarlyModLoads && !CACHED_MOD) {
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
       sv[k] = load_vec(sr, tid + k * T, p.stream_mask & kScale);
@@ -536,7 +543,7 @@ fused_norm_rows(const RowParams p) {
     }
   }
 
-  if (!FN_EARLY_MODULATION_LOADS && !CACHED_MOD) {
+  if (!RowShape<D>::kEarlyModLoads && !CACHED_MOD) {
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
       sv[k] = load_vec(sr, tid + k * T, p.stream_mask & kScale);
