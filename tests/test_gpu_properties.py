@@ -264,3 +264,47 @@ def test_near_cancellation_and_offsets_bit_exact(is_rms, offset, spread):
     print(f"\nnear-cancellation offset={offset} spread={spread} rms={is_rms}\n  y: {ty}\n  r: {tr}")
     assert tr.exact == tr.n
     assert ty.hist.get(0, 0) == ty.n, f"y not bit-exact: {ty}"
+
+
+@pytest.mark.parametrize("D", [5120, 10240])
+@pytest.mark.parametrize("op", ["fused", "norm_only"])
+@pytest.mark.parametrize("is_rms", [False, True])
+@pytest.mark.parametrize("offset,spread", [(1000.0, 1.0), (1000.0, 0.01), (-3.0e4, 1.0), (0.0, 1e-3)])
+def test_offset_rows_with_broadcast_modulation_bit_exact(D, op, is_rms, offset, spread):
+    # broadcast scale and shift run the instances that re-read them from cache (for
+    # norm-only at D=10240 with 256 threads per row); rows whose mean dwarfs their spread
+    # take the centred second pass, which re-reads the row from memory
+    from helpers import f32_to_bf16_bits_rne
+    L = 40
+    rng = np.random.default_rng(7 + D + int(is_rms))
+    bfbits = lambda a: f32_to_bf16_bits_rne(np.asarray(a, dtype=np.float32))
+    base = bfbits(offset + spread * rng.normal(size=(1, L, D)))
+    x = bfbits(rng.normal(size=(1, L, D))) if op == "fused" else base
+    gate = bfbits(0.5 * rng.normal(size=(1, 1, D)))
+    scale = bfbits(0.3 * rng.normal(size=(1, 1, D)))
+    shift = bfbits(0.1 * rng.normal(size=(1, 1, D)))
+    weight = bfbits(1 + 0.1 * rng.normal(size=D))
+    dev = lambda a: from_bits(a, DEV)
+    norm = "rms" if is_rms else "layer"
+    st, b0 = (L * D, 0, D), (0, 0, 0)
+    if op == "fused":
+        y, r = fn.fused_residual_norm_scale_shift(dev(base), dev(x), dev(gate), dev(weight), None,
+                                                  dev(scale), dev(shift), norm, 1e-6)
+        ref = oracle.fused_norm(1, L, D, x=x, x_st=st, residual=base, res_st=st, gate=gate, gate_st=b0,
+                                weight=weight, scale=scale, scale_st=b0, shift=shift, shift_st=b0,
+                                is_rms=is_rms)
+    else:
+        y = fn.norm_scale_shift(dev(x), dev(weight), None, dev(scale), dev(shift), norm, 1e-6)
+        r = None
+        ref = oracle.fused_norm(1, L, D, x=x, x_st=st, weight=weight, scale=scale, scale_st=b0,
+                                shift=shift, shift_st=b0, is_rms=is_rms, norm_only=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(y), ref["y"]), "y not bit-exact"
+    if r is not None:
+        assert np.array_equal(bits(r), ref["r"]), "r not bit-exact"
+    if (offset, spread) == (1000.0, 1.0) and not is_rms:
+        # the case is built so that some rows take the centred pass (mean^2 > 2^20 var > 0)
+        from helpers import bf16_bits_to_f64
+        v = bf16_bits_to_f64(ref["r"] if r is not None else x).reshape(L, D)
+        mu, var = v.mean(axis=1), v.var(axis=1)
+        assert np.any((mu * mu > 2.0 ** 20 * var) & (var > 0))
