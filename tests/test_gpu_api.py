@@ -1,11 +1,14 @@
-"""GPU checks of the launch contract: which error a launch reports, and which device it
-runs on.
+"""GPU checks of the launch contract: which error a launch reports, which device it runs
+on, that each call runs the CUDA kernel, and that one handle serves every launch shape.
 
 * fused_norm_launch reports the status of its own launch only. An error left pending in
   the caller's CUDA runtime (here: torch's, by an invalid cudaSetDevice, a host-side
   argument error that touches no GPU) is neither returned as FN_ERR_CUDA nor cleared.
 * The tensor-level API runs on its inputs' device whichever device is current (needs
   two GPUs; skipped otherwise).
+* A CUDA activity trace shows exactly one fused_norm_rows kernel per call, nothing else.
+* One handle launched with different L, frame counts and operand layouts matches the
+  oracle bit for bit each time.
 """
 import ctypes
 
@@ -91,3 +94,67 @@ def test_api_runs_on_the_inputs_device():
     assert torch.equal(y.view(torch.int16), want_y.view(torch.int16))
     assert torch.equal(r.view(torch.int16), want_r.view(torch.int16))
     assert torch.equal(n.view(torch.int16), want_n.view(torch.int16))
+
+
+def test_every_call_runs_the_cuda_kernel():
+    # the pages' tests count dispatches to prove there is no silent fallback; here the
+    # CUDA activity trace of a few calls must show exactly one fused_norm_rows kernel per
+    # call and nothing else
+    try:
+        from torch.profiler import ProfilerActivity, profile
+    except ImportError:
+        pytest.skip("torch.profiler unavailable")
+    dev = torch.device("cuda:0")
+    B, L, D = 1, 96, 5120
+    x, res = _rand((B, L, D), 21, dev), _rand((B, L, D), 22, dev)
+    gate, scale, shift = (_rand((1, 1, D), s, dev, 0.1) for s in (23, 24, 25))
+    y = torch.empty_like(x)
+    r = torch.empty_like(x)
+    n = torch.empty_like(x)
+    torch.cuda.synchronize(dev)
+    calls = 3
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        for _ in range(calls):
+            fn.fused_residual_norm_scale_shift(res, x, gate, None, None, scale, shift, "layer", 1e-6,
+                                               out=y, residual_out=r)
+            fn.norm_scale_shift(x, None, None, scale, shift, "rms", 1e-6, out=n)
+        torch.cuda.synchronize(dev)
+    kernels = [e.name for e in prof.events() if e.device_type.name == "CUDA"]
+    if not kernels:
+        pytest.skip("no CUDA activity recorded (tracing unavailable)")
+    ours = [k for k in kernels if "fused_norm_rows" in k]
+    assert len(ours) == 2 * calls, kernels
+    assert len(kernels) == len(ours), kernels
+
+
+def test_one_handle_serves_every_length_and_layout():
+    # a handle fixes only the specialisation; L, B, frames and operand strides are launch
+    # arguments (the pages test that one compiled kernel is reused across L and layouts)
+    import numpy as np
+    import synth
+    from parity import Tally, compare_rows, host_inputs, upload_host
+    dev = torch.device("cuda:0")
+    cfg = _abi.fn_config(D=5120, is_rms=0, has_gate=1, has_weight=1, has_bias=0, norm_only=0,
+                         affine_fp32=0, eps=1e-6)
+    st, h = _abi.fused_norm_create(cfg)
+    assert st == fn.FN_OK
+    spec = synth.Spec(False, True, True)
+    try:
+        for L, F, layouts in ((16, 0, ("bcast", "row", "row")), (531, 9, ("frame", "frame", "frame")),
+                              (1237, 0, ("row", "bcast", "bcast"))):
+            w = synth.dataclasses.replace(synth.scaled(synth.W3, L), F=F,
+                                          layouts=(("gate", layouts[0]), ("scale", layouts[1]),
+                                                   ("shift", layouts[2])), name=f"reuse_L{L}")
+            host = host_inputs(w)
+            d = upload_host(w, host, dev)
+            y = torch.empty((w.B, w.L, w.D), dtype=torch.bfloat16, device=dev)
+            r = torch.empty_like(y)
+            args = fn.build_args(d["x"], d["residual"], d["gate"], d["weight"], None, d["scale"],
+                                 d["shift"], y, r)
+            assert _abi.fused_norm_launch(h, args, int(torch.cuda.current_stream(dev).cuda_stream)) == fn.FN_OK
+            torch.cuda.synchronize(dev)
+            ty, tr = Tally(), Tally()
+            compare_rows(w, spec, y, r, np.arange(w.rows), ty, tr, host=host)
+            assert ty.exact == ty.n and tr.exact == tr.n, (L, layouts, str(ty), str(tr))
+    finally:
+        _abi.fused_norm_destroy(h)
