@@ -774,10 +774,10 @@ def free_port():
 
 def launch_ranks(args):
     """`--gpus N` (N > 1) without a torchrun environment: start the N ranks under
-    torch.distributed.run on this node and return their exit status. Each rank's
-    OpenMP pool gets its share of the host cores."""
+    torch.distributed.run on this node and return their exit status. Host-side work
+    (generating the node-shared inputs, the CPU legs) runs on local rank 0 alone, so
+    every rank keeps the whole host's OpenMP pool."""
     env = dict(os.environ)
-    env.setdefault("OMP_NUM_THREADS", str(max(1, (os.cpu_count() or 1) // args.gpus)))
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
            f"--nproc-per-node={args.gpus}", "--master-addr=127.0.0.1", f"--master-port={free_port()}",
            os.path.abspath(__file__), *sys.argv[1:]]
