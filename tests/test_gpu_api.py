@@ -9,6 +9,7 @@ on, that each call runs the CUDA kernel, and that one handle serves every launch
 * A CUDA activity trace shows exactly one fused_norm_rows kernel per call, nothing else.
 * One handle launched with different L, frame counts and operand layouts matches the
   oracle bit for bit each time.
+* Launches captured into a CUDA graph replay to the eager results.
 """
 import ctypes
 
@@ -158,3 +159,31 @@ def test_one_handle_serves_every_length_and_layout():
             assert ty.exact == ty.n and tr.exact == tr.n, (L, layouts, str(ty), str(tr))
     finally:
         _abi.fused_norm_destroy(h)
+
+
+def test_launches_replay_from_a_cuda_graph():
+    # the library launches on the caller's stream and allocates nothing, so its launches
+    # can be captured into a CUDA graph and replayed; the replay gives the eager bits
+    dev = torch.device("cuda:0")
+    B, L, D = 2, 40, 5120
+    x, res = _rand((B, L, D), 31, dev), _rand((B, L, D), 32, dev)
+    gate, scale, shift = _rand((B, L, D), 33, dev, 0.5), _rand((1, D), 34, dev, 0.1), _rand((1, D), 35, dev, 0.1)
+    weight = (1 + _rand((D,), 36, dev, 0.1).float()).to(torch.bfloat16)
+    want_y, want_r = fn.fused_residual_norm_scale_shift(res, x, gate, weight, None, scale, shift, "rms")
+    want_n = fn.norm_scale_shift(x, weight, None, scale, shift, "layer")
+    y, r, n = torch.empty_like(x), torch.empty_like(x), torch.empty_like(x)
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(cap), torch.cuda.graph(graph, stream=cap):
+        fn.fused_residual_norm_scale_shift(res, x, gate, weight, None, scale, shift, "rms", out=y,
+                                           residual_out=r, stream=cap)
+        fn.norm_scale_shift(x, weight, None, scale, shift, "layer", out=n, stream=cap)
+    for _ in range(2):
+        y.zero_(), r.zero_(), n.zero_()
+        graph.replay()
+        torch.cuda.synchronize(dev)
+        for got, want in ((y, want_y), (r, want_r), (n, want_n)):
+            assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+    del graph
