@@ -2,7 +2,8 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--spec NAME] [--rows L] [--graph | --flush-l2]
-                    [--no-e2e] [--no-cpu-baseline] [--e2e-steps E] [--cpu-seconds S]
+                    [--affine-fp32] [--dit-mix] [--no-e2e] [--no-cpu-baseline]
+                    [--e2e-steps E] [--cpu-seconds S]
 
 One step = one call of the op over the whole workload (every full tensor read or
 written once). Default workload: WAN2.2-shaped LayerNorm, B=1 L=176400 D=5120 bf16,
@@ -71,6 +72,10 @@ def parse():
     p.add_argument("--affine-fp32", action="store_true",
                    help="weight and bias as fp32 (used at full precision), as the pages' "
                         "microbenchmark passes them")
+    p.add_argument("--dit-mix", action="store_true",
+                   help="one step = the norm calls of one WAN2.2 DiT forward on the pages' "
+                        "microbenchmark shape: 41 norm_scale_shift, 40 fused without affine, 40 "
+                        "fused with fp32 weight and bias (use with a small --steps)")
     p.add_argument("--graph", action="store_true",
                    help="replay the timed launches from one CUDA graph (removes host launch "
                         "overhead; for the launch-bound small shapes)")
@@ -253,6 +258,9 @@ def run_ours(args):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
 
+    if args.dit_mix:   # inputs for all three ops of the mix: fused with fp32 w and b reads them all
+        args.workload, args.spec, args.affine_fp32 = "microbench_bcast_B1_L176400_D5120", "ln_gate_w_b", True
+        args.no_e2e = args.no_cpu_baseline = True
     w = workload(args)
     spec = pick_spec(w, args)
     bytes_step = w.algorithmic_bytes(spec)
@@ -291,10 +299,28 @@ def run_ours(args):
     handle = fn.api._handle(w.D, spec.is_rms, spec.has_gate, spec.has_weight, spec.has_bias,
                             spec.norm_only, w.eps, affine_fp32)
 
+    # (handle, C arguments, launches per step); one step launches each of them that often
+    calls = [(handle, args_c, 1)]
+    mix = None
+    if args.dit_mix:
+        nss = synth.Spec(False, False, False, norm_only=True)
+        fused = synth.Spec(False, True, False)
+        h_nss = fn.api._handle(w.D, False, False, False, False, True, w.eps, False)
+        h_fused = fn.api._handle(w.D, False, True, False, False, False, w.eps, False)
+        a_nss = fn.build_args(d["x"], None, None, None, None, d["scale"], d["shift"], y, None)
+        a_fused = fn.build_args(d["x"], d["residual"], d["gate"], None, None, d["scale"], d["shift"], y, r)
+        calls = [(h_nss, a_nss, 41), (h_fused, a_fused, 40), (handle, args_c, 40)]
+        bytes_step = 41 * w.algorithmic_bytes(nss) + 40 * w.algorithmic_bytes(fused) + 40 * bytes_step
+        mix = {"norm_scale_shift (LN, no affine)": 41, "fused (LN, gate, no affine)": 40,
+               "fused (LN, gate, fp32 weight and bias)": 40}
+    per_step = sum(c[2] for c in calls)
+
     def step():
-        st = fn.fused_norm_launch(handle, args_c, int(stream.cuda_stream))
-        if st != fn.FN_OK:
-            raise fn.FusedNormError(st, "fused_norm_launch", fn.fused_norm_status_string(st))
+        for h_, a_, count in calls:
+            for _ in range(count):
+                st = fn.fused_norm_launch(h_, a_, int(stream.cuda_stream))
+                if st != fn.FN_OK:
+                    raise fn.FusedNormError(st, "fused_norm_launch", fn.fused_norm_status_string(st))
 
     # one call through the tensor-level API first: same result as the prebuilt launch
     if spec.norm_only:
@@ -351,19 +377,19 @@ def run_ours(args):
     if graph is not None:
         with torch.cuda.stream(stream):
             graph.replay()
-        launches = K
+        launches = K * per_step
         ev[K].record(stream)
     elif scratch is not None:
         for i in range(K):
             scratch.zero_()           # 512 MB written: the inputs leave the 126 MB L2
             starts[i].record(stream)
             step()
-            launches += 1
+            launches += per_step
             ev[i + 1].record(stream)
     else:
         for i in range(K):
             step()
-            launches += 1
+            launches += per_step
             ev[i + 1].record(stream)
     torch.cuda.synchronize(dev)
     barrier()
@@ -404,15 +430,18 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded normal draws, WAN2.2 shapes; no model weights)",
             "config": dict(config_dict(w, spec, world, affine_fp32), launch="cuda_graph" if graph is not None else "stream",
+                           **({"workload": f"dit_forward_mix_{w.name}", "calls_per_step": mix,
+                               "spec": None} if mix else {}),
                            **({"l2": "flushed before every timed launch (512 MB write, outside the "
                                      "per-launch events)"} if scratch is not None else {})),
-            "rows_per_s": round(world * w.rows / (ms_step * 1e-3), 1),
+            "rows_per_s": round(world * w.rows * per_step / (ms_step * 1e-3), 1),
             "pct_of_peak": round(100.0 * value / world / peak, 2),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                          "peak_kind": f"{peak_kind} (HBM copy bandwidth)", "unit": "GB/s",
                          "frac": round(achieved / peak, 4),
                          "traffic": recorded_traffic(w, spec), "kernel": KERNEL,
-                         "algorithmic_bytes_per_launch": bytes_step,
+                         "algorithmic_bytes_per_launch": bytes_step // per_step if per_step == 1 else None,
+                         "algorithmic_bytes_per_step": bytes_step, "launches_per_step": per_step,
                          "kernel_ms_mean": round(kernel_ms, 5),
                          "kernel_ms_median": round(statistics.median(per), 5)},
             "clocks": clocks,

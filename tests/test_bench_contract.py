@@ -83,3 +83,14 @@ def test_kernel_digest_ignores_comments_only():
     assert bench._code_tokens(base) != bench._code_tokens(base.replace("a + b", "a - b"))
     assert bench._code_tokens(base) != bench._code_tokens(base.replace("// not a", "// NOT a"))
     assert bench._code_tokens("c = '\\''; // q") == "c = '\\'';"
+
+
+@pytest.mark.gpu
+def test_gpu_arm_dit_forward_mix():
+    # one step = the 121 norm calls of a DiT forward (41 + 40 + 40) on the broadcast shape
+    d = _run(["--dit-mix", "--rows", "4096", "--steps", "2", "--warmup", "3"])
+    assert d["gpu_launches"] == 2 * 121
+    assert sum(d["config"]["calls_per_step"].values()) == 121
+    assert d["config"]["workload"].startswith("dit_forward_mix")
+    assert d["roofline"]["launches_per_step"] == 121 and d["value"] > 0
+    assert d["e2e"] is None and d["cpu_baseline"] is None
