@@ -26,9 +26,9 @@
 //     the same bf16 value, so does the exact value (rounding is monotone), and that is
 //     the result. Otherwise (a few in 10^4 elements) the element is recomputed in fp64
 //     and rounded once (round-to-odd to fp32, then nearest-even to bf16). y is therefore
-//     the correctly rounded bf16 of the formula evaluated with the fp64 statistics
-//     (up to the fp64 evaluation's own last-bit error). The fp32 arithmetic can run two
-//     elements per instruction (sm_100 f32x2), with results identical to the scalar form.
+//     the bf16 rounding of the formula evaluated in fp64 with the fp64 statistics, within
+//     one bf16 ulp of the exact value. The fp32 arithmetic runs two elements per
+//     instruction where it can (sm_100 f32x2), with results identical to the scalar form.
 //   * r is the correctly rounded bf16 of the exact residual + gate * x: one bf16x2
 //     fused multiply-add per pair computes the exact value and rounds it once.
 //   * Per-row (streamed-once) operands use evict-first loads and stores; broadcast
