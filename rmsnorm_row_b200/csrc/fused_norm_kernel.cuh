@@ -189,6 +189,7 @@ __device__ __forceinline__ double div_by_row_length(double a) {
   static_assert(D == 5120 || D == 10240, "D must be 5 * 2^k");
   constexpr double kScale = D == 5120 ? 1.0 / 1024.0 : 1.0 / 2048.0;
   const double q0 = __dmul_rn(a, 0.2);
+  if (!isfinite(q0)) return q0 * kScale;  // an infinite or NaN sum divides to itself
   const double r = fma(-5.0, q0, a);
   return fma(r, 0.2, q0) * kScale;
 }
@@ -587,7 +588,8 @@ fused_norm_rows(const RowParams p) {
     st.rho = rsqrt(div_by_row_length<D>(t2) + p.eps);
   } else {
     const double mu = div_by_row_length<D>(t1);
-    double var = fmax(div_by_row_length<D>(t2) - mu * mu, 0.0);
+    double var = div_by_row_length<D>(t2) - mu * mu;
+    if (var < 0.0) var = 0.0;  // rounding below zero; a NaN (non-finite row) stays NaN
     if (mu * mu > 1048576.0 * var && var > 0.0) {
       // The mean dwarfs the spread: take the variance around the mean instead
       // (uniform branch: every thread of the CTA has the same statistics). The row

@@ -308,3 +308,52 @@ def test_offset_rows_with_broadcast_modulation_bit_exact(D, op, is_rms, offset, 
         v = bf16_bits_to_f64(ref["r"] if r is not None else x).reshape(L, D)
         mu, var = v.mean(axis=1), v.var(axis=1)
         assert np.any((mu * mu > 2.0 ** 20 * var) & (var > 0))
+
+
+@pytest.mark.parametrize("D", [5120, 10240])
+@pytest.mark.parametrize("is_rms", [False, True])
+def test_special_values_propagate_like_the_oracle(D, is_rms):
+    # IEEE propagation with no special handling: a NaN in x, an infinity in the residual
+    # and a residual + gate * x that overflows bf16 poison their own rows (r at that
+    # element; y through the statistics: all NaN for a NaN, and for LayerNorm's
+    # inf - inf; RMSNorm's 1/sqrt(inf) = 0 leaves y = shift but inf * 0 at the element);
+    # the other rows are untouched. NaN payloads may differ, so NaN positions are
+    # compared as a mask and every other element bit for bit.
+    from helpers import f32_to_bf16_bits_rne
+    L = 8
+    rng = np.random.default_rng(99 + D)
+    bfbits = lambda a: f32_to_bf16_bits_rne(np.asarray(a, dtype=np.float32))
+    res = bfbits(rng.normal(size=(1, L, D)))
+    x = bfbits(rng.normal(size=(1, L, D)))
+    gate = bfbits(0.5 * rng.normal(size=(1, 1, D)))
+    scale = bfbits(0.1 * rng.normal(size=(1, L, D)))
+    shift = bfbits(0.1 * rng.normal(size=(1, L, D)))
+    x[0, 0, 17] = 0x7FC0                      # NaN
+    res[0, 1, 3] = 0x7F80                     # +inf
+    gate[0, 0, 5] = 0x3F80                    # 1.0
+    res[0, 2, 5] = x[0, 2, 5] = 0x7F7F        # bf16 max: the sum overflows to +inf
+    dev = lambda a: from_bits(a, DEV)
+    y, r = fn.fused_residual_norm_scale_shift(dev(res), dev(x), dev(gate), None, None, dev(scale),
+                                              dev(shift), "rms" if is_rms else "layer", 1e-6)
+    torch.cuda.synchronize()
+    st = (L * D, 0, D)
+    ref = oracle.fused_norm(1, L, D, x=x, x_st=st, residual=res, res_st=st, gate=gate,
+                            gate_st=(0, 0, 0), scale=scale, scale_st=st, shift=shift, shift_st=st,
+                            is_rms=is_rms)
+
+    def nan_mask(b):
+        b = np.asarray(b, dtype=np.uint16)
+        return ((b & 0x7F80) == 0x7F80) & ((b & 0x7F) != 0)
+
+    for got, want in ((bits(y), ref["y"]), (bits(r), ref["r"])):
+        got, want = got.reshape(L, D), want.reshape(L, D)
+        assert np.array_equal(nan_mask(got), nan_mask(want))
+        keep = ~nan_mask(want)
+        assert np.array_equal(got[keep], want[keep])
+    ry = bits(y).reshape(L, D)
+    assert nan_mask(ry[0]).all()              # a NaN reaches every statistic
+    if not is_rms:
+        assert nan_mask(ry[1:3]).all()        # inf - inf in the variance
+    assert not nan_mask(ry[3:]).any()         # the other rows are finite
+    rr = bits(r).reshape(L, D)
+    assert rr[1, 3] == 0x7F80 and rr[2, 5] == 0x7F80 and nan_mask(rr[0, 17])
