@@ -357,3 +357,27 @@ def test_special_values_propagate_like_the_oracle(D, is_rms):
     assert not nan_mask(ry[3:]).any()         # the other rows are finite
     rr = bits(r).reshape(L, D)
     assert rr[1, 3] == 0x7F80 and rr[2, 5] == 0x7F80 and nan_mask(rr[0, 17])
+
+
+@pytest.mark.parametrize("D", [5120, 10240])
+@pytest.mark.parametrize("is_rms", [False, True])
+def test_zero_spread_with_zero_eps_matches_the_oracle(D, is_rms):
+    # eps = 0 on rows with no spread (LayerNorm: a constant row; RMSNorm: a zero row):
+    # 1/sqrt(0) = inf and 0 * inf = NaN on both sides; rows with spread stay finite
+    from helpers import f32_to_bf16_bits_rne
+    L = 4
+    rng = np.random.default_rng(5 + D)
+    bfbits = lambda a: f32_to_bf16_bits_rne(np.asarray(a, dtype=np.float32))
+    x = bfbits(rng.normal(size=(1, L, D)))
+    x[0, 0, :] = 0x0000 if is_rms else 0x4040    # 0.0 or 3.0 across the row
+    scale = bfbits(0.1 * rng.normal(size=(1, 1, D)))
+    shift = bfbits(0.1 * rng.normal(size=(1, 1, D)))
+    dev = lambda a: from_bits(a, DEV)
+    y = fn.norm_scale_shift(dev(x), None, None, dev(scale), dev(shift), "rms" if is_rms else "layer", 0.0)
+    torch.cuda.synchronize()
+    ref = oracle.fused_norm(1, L, D, x=x, x_st=(L * D, 0, D), scale=scale, scale_st=(0, 0, 0),
+                            shift=shift, shift_st=(0, 0, 0), is_rms=is_rms, norm_only=True, eps=0.0)
+    got, want = bits(y).reshape(L, D), ref["y"].reshape(L, D)
+    nan = lambda b: ((b & 0x7F80) == 0x7F80) & ((b & 0x7F) != 0)
+    assert nan(want[0]).all() and nan(got[0]).all()
+    assert np.array_equal(got[1:], want[1:])
