@@ -32,7 +32,7 @@ def exact_bits(vals):
     """bf16 bit patterns of values that must be exactly representable in bf16."""
     f = np.asarray(vals, dtype=np.float64)
     b = f32_to_bf16_bits_rne(f.astype(np.float32))
-    assert np.array_equal(bf16_bits_to_f64(b), f), "value not exact in bf16"
+    assert np.array_equal(bf16_bits_to_f64(b), f, equal_nan=True), "value not exact in bf16"
     return b
 
 
@@ -136,6 +136,39 @@ def test_bf16_rne_specials():
     assert oracle.bf16_rne(2.0 ** -134) == 0x0000          # tie -> even (zero)
     assert oracle.bf16_rne(2.0 ** -134 * (1 + 2**-20)) == 0x0001
     assert oracle.bf16_rne(-3 * 2.0 ** -134) == 0x8002     # tie between 1 and 2 quanta -> 2
+
+
+def test_special_values_follow_ieee():
+    # c15: no special handling. A NaN reaches every statistic of its row; an infinity
+    # gives LayerNorm inf - inf (NaN everywhere) but RMSNorm 1/sqrt(inf) = 0, so each
+    # finite element's n is exactly 0 and y = shift, and the infinite element 0 * inf = NaN
+    D = 16
+    nan = lambda b: ((np.asarray(b) & 0x7F80) == 0x7F80) & ((np.asarray(b) & 0x7F) != 0)
+    rng = np.random.default_rng(3)
+    vals = exact_bits(np.round(rng.normal(size=D) * 8) / 8)
+    shift = np.round(rng.normal(size=D) * 16) / 64
+    scale = np.round(rng.normal(size=D) * 16) / 64
+    for is_rms in (False, True):
+        res = bf16_bits_to_f64(vals).copy()
+        res[3] = np.nan
+        out = one_row(res, scale=scale, shift=shift, is_rms=is_rms)
+        assert nan(out["y"]).all() and nan(out["r"][0, 0, 3])
+    res = bf16_bits_to_f64(vals).copy()
+    res[5] = np.inf
+    out = one_row(res, scale=scale, shift=shift, is_rms=False)
+    assert nan(out["y"]).all() and out["r"][0, 0, 5] == 0x7F80
+    out = one_row(res, scale=scale, shift=shift, is_rms=True)
+    y = out["y"].reshape(-1)
+    assert nan(y[5])
+    keep = np.arange(D) != 5
+    assert np.array_equal(y[keep], exact_bits(shift)[keep])
+    # an overflowing residual + gate * x is an infinity in r
+    big = float(Fraction(2**127) * (2 - Fraction(1, 128)))   # bf16 max
+    res = bf16_bits_to_f64(vals).copy()
+    xs = np.zeros(D)
+    res[7], xs[7] = big, big
+    out = one_row(res, x_vals=xs, gate_vals=np.ones(D), scale=scale, shift=shift, is_rms=True)
+    assert out["r"][0, 0, 7] == 0x7F80 and nan(out["y"][0, 0, 7])
 
 
 # --------------------------------------------------------------------------
