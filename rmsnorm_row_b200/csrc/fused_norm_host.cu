@@ -244,10 +244,11 @@ fn_status fused_norm_create(fused_norm_t* out, const fn_config* cfg) {
   h->cfg = c;
   h->launch = fn;
   h->launch_cached_mod = fn_cm;
-  h->threads = c.D / (8 * (c.D == 5120 ? RowShape<5120>::VPT : RowShape<10240>::VPT));
-  const int vpt_cm = c.norm_only ? (c.D == 5120 ? RowShape<5120>::kVptNss : RowShape<10240>::kVptNss)
-                                 : (c.D == 5120 ? RowShape<5120>::kVptCachedMod : RowShape<10240>::kVptCachedMod);
-  h->threads_cached_mod = c.D / (8 * vpt_cm);
+  const bool affine = c.has_weight || c.has_bias;
+  for (int cm = 0; cm < 2; ++cm) {
+    const int vpt = c.D == 5120 ? vpt_of<5120>(c.norm_only, cm, affine) : vpt_of<10240>(c.norm_only, cm, affine);
+    (cm ? h->threads_cached_mod : h->threads) = c.D / (8 * vpt);
+  }
   *out = h;
   return FN_OK;
 }

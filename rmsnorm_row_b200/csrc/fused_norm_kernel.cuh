@@ -433,28 +433,48 @@ template <int D> struct RowShape;
 #define FN_EARLY_MODULATION_LOADS_10240 1
 #endif
 // Norm-only with broadcast / per-frame scale and shift reads one tensor and writes one
-// per row, so its per-element arithmetic, not HBM, sets its pace: those instances run
-// 8 CTAs per SM at D = 5120 (64 registers, no spills; measured 3% faster than 7, which was
-// 1% faster than 6).
-#ifndef FN_MINB_NSS_5120
-#define FN_MINB_NSS_5120 8
-#endif
+// per row, so its per-element arithmetic and the latency of each row's statistics, not
+// HBM, set its pace. Without weight or bias those instances hold 10 vectors per thread:
+// fewer threads per row share the per-thread fixed work (the reduction tail, the fp64
+// division and square root, the row addressing), and more rows are in flight per SM.
+// D = 5120: 64 threads, 12 CTAs per SM (80 registers, no spills); D = 10240: 128 threads,
+// 6 CTAs per SM. Measured on B200 against 128 x 5 at 8 CTAs (D = 5120) and 256 x 5 at 4
+// (D = 10240): broadcast LayerNorm 6% and 10% faster, per-frame 2% and 5%. One warp per
+// row (20 vectors per lane, 16 warps per SM) was 24% slower at D = 5120: fewer
+// instructions, but too few rows in flight.
+// With weight or bias (more cached operands per vector) the 64 x 10 shape measured 10%
+// slower at D = 5120 (LayerNorm, bf16 weight and bias), so those keep 128 x 5 at 8 CTAs;
+// at D = 10240 they take 128 x 10 as well (RMSNorm with weight 4% faster than 256 x 5),
+// fp32 affine values at one CTA fewer (2% faster; with 6 CTAs they spill and are slower).
 #ifndef FN_VPT_NSS_5120
-#define FN_VPT_NSS_5120 FN_VPT_5120
+#define FN_VPT_NSS_5120 10
 #endif
-// At D = 10240 they take 256 threads x 5 vectors at 4 CTAs per SM instead of 320 x 4 at
-// 3: measured 0.79 -> 0.69 ms on a broadcast norm-only shape (L = 90000). The fused
-// instances with cached modulation keep 320 x 4 (256 x 5 is mixed there: -2% to +3%).
-#ifndef FN_MINB_NSS_10240
-#define FN_MINB_NSS_10240 4
+#ifndef FN_MINB_NSS_5120
+#define FN_MINB_NSS_5120 12
+#endif
+#ifndef FN_VPT_NSS_AFFINE_5120
+#define FN_VPT_NSS_AFFINE_5120 5
+#endif
+#ifndef FN_MINB_NSS_AFFINE_5120
+#define FN_MINB_NSS_AFFINE_5120 8
 #endif
 #ifndef FN_VPT_NSS_10240
-#define FN_VPT_NSS_10240 5
+#define FN_VPT_NSS_10240 10
+#endif
+#ifndef FN_MINB_NSS_10240
+#define FN_MINB_NSS_10240 6
+#endif
+#ifndef FN_VPT_NSS_AFFINE_10240
+#define FN_VPT_NSS_AFFINE_10240 10
+#endif
+#ifndef FN_MINB_NSS_AFFINE_10240
+#define FN_MINB_NSS_AFFINE_10240 6
 #endif
 template <> struct RowShape<5120> {
   static constexpr int VPT = FN_VPT_5120, kMinBlocks = FN_MINB_5120;
   static constexpr int kMinBlocksCachedMod = FN_MINB_CM_5120, kVptCachedMod = FN_VPT_CM_5120;
   static constexpr int kMinBlocksNss = FN_MINB_NSS_5120, kVptNss = FN_VPT_NSS_5120;
+  static constexpr int kMinBlocksNssAffine = FN_MINB_NSS_AFFINE_5120, kVptNssAffine = FN_VPT_NSS_AFFINE_5120;
   static constexpr bool kPaired = FN_PAIRED_5120 != 0;
   static constexpr bool kEarlyModLoads = FN_EARLY_MODULATION_LOADS_5120 != 0;
 };
@@ -462,28 +482,43 @@ template <> struct RowShape<10240> {
   static constexpr int VPT = FN_VPT_10240, kMinBlocks = FN_MINB_10240;
   static constexpr int kMinBlocksCachedMod = FN_MINB_CM_10240, kVptCachedMod = FN_VPT_CM_10240;
   static constexpr int kMinBlocksNss = FN_MINB_NSS_10240, kVptNss = FN_VPT_NSS_10240;
+  static constexpr int kMinBlocksNssAffine = FN_MINB_NSS_AFFINE_10240, kVptNssAffine = FN_VPT_NSS_AFFINE_10240;
   static constexpr bool kPaired = FN_PAIRED_10240 != 0;
   static constexpr bool kEarlyModLoads = FN_EARLY_MODULATION_LOADS_10240 != 0;
 };
+
+// Vectors per thread of an instance (its CTA has D / (8 VPT) threads): by operand
+// placement (norm-only, scale and shift cached) and whether it has a weight or bias.
+// The launchers and the host's launch plan both take the shape from here.
+template <int D>
+__host__ __device__ constexpr int vpt_of(bool norm_only, bool cached_mod, bool affine) {
+  return (norm_only && cached_mod) ? (affine ? RowShape<D>::kVptNssAffine : RowShape<D>::kVptNss)
+         : cached_mod              ? RowShape<D>::kVptCachedMod
+                                   : RowShape<D>::VPT;
+}
 
 // CTAs per SM an instance's register budget is sized for. The figure is per D and
 // operand placement: instances that carry more live values (fp32 affine, bias, RMSNorm
 // with weight at D = 10240) spill a few registers to L1 at these counts, and most measured
 // faster so than with one CTA fewer (D = 10240, broadcast modulation: 1.15 ms with 3 CTAs
-// per SM and spills, 1.30 ms with 2 and none). The exception is an fp32 bias with cached
+// per SM and spills, 1.30 ms with 2 and none). The exceptions are an fp32 bias with cached
 // modulation, whose 16 fp32 affine values per vector spill ~90 bytes at 6 CTAs: one CTA
 // fewer is 4% faster there (the pages' broadcast shape with fp32 w and b), while fp32
-// weight alone is 2% slower with one CTA fewer.
-template <int D, bool NORM_ONLY, bool CACHED_MOD, bool AFFINE_F32, bool HAS_BIAS>
+// weight alone is 2% slower with one CTA fewer; and norm-only fp32 affine at D = 10240
+// (above).
+template <int D, bool NORM_ONLY, bool CACHED_MOD, bool AFFINE_F32, bool HAS_WEIGHT, bool HAS_BIAS>
 constexpr int min_blocks() {
-  return (NORM_ONLY && CACHED_MOD) ? RowShape<D>::kMinBlocksNss
+  return (NORM_ONLY && CACHED_MOD)
+             ? ((HAS_WEIGHT || HAS_BIAS)
+                    ? RowShape<D>::kMinBlocksNssAffine - ((AFFINE_F32 && D == 10240) ? 1 : 0)
+                    : RowShape<D>::kMinBlocksNss)
          : CACHED_MOD ? RowShape<D>::kMinBlocksCachedMod - ((AFFINE_F32 && HAS_BIAS && D == 5120) ? 1 : 0)
                       : RowShape<D>::kMinBlocks;
 }
 
 template <int D, int VPT, bool IS_RMS, bool NORM_ONLY, bool HAS_GATE, bool HAS_WEIGHT, bool HAS_BIAS,
           bool AFFINE_F32, bool CACHED_MOD>
-__global__ void __launch_bounds__(D / (8 * VPT), (min_blocks<D, NORM_ONLY, CACHED_MOD, AFFINE_F32, HAS_BIAS>()))
+__global__ void __launch_bounds__(D / (8 * VPT), (min_blocks<D, NORM_ONLY, CACHED_MOD, AFFINE_F32, HAS_WEIGHT, HAS_BIAS>()))
 fused_norm_rows(const RowParams p) {
   constexpr int T = D / (8 * VPT);
   constexpr int W = T / 32;
@@ -658,8 +693,9 @@ cudaError_t launch_rows(const RowParams& p, int64_t grid, cudaStream_t stream) {
 // Launcher for one (norm_only, gate, modulation caching) group: the affine combinations.
 template <int D, bool RMS, bool NO, bool G, bool CM>
 LaunchFn pick_affine(bool w, bool b, bool f32) {
-  constexpr int V = (NO && CM) ? RowShape<D>::kVptNss : CM ? RowShape<D>::kVptCachedMod : RowShape<D>::VPT;
-  if (!w && !b) return &launch_rows<D, V, RMS, NO, G, false, false, false, CM>;
+  constexpr int V0 = vpt_of<D>(NO, CM, false);  // no weight or bias
+  constexpr int V = vpt_of<D>(NO, CM, true);
+  if (!w && !b) return &launch_rows<D, V0, RMS, NO, G, false, false, false, CM>;
   if (f32) {
     if (w && b) return &launch_rows<D, V, RMS, NO, G, true, true, true, CM>;
     return w ? &launch_rows<D, V, RMS, NO, G, true, false, true, CM>

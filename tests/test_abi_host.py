@@ -149,18 +149,21 @@ def test_valid_args_pass_and_plan():
 @pytest.mark.parametrize("D", [5120, 10240])
 @pytest.mark.parametrize("norm_only", [0, 1])
 @pytest.mark.parametrize("bcast", [False, True])
-def test_plan_follows_the_instance(D, norm_only, bcast):
+@pytest.mark.parametrize("weight", [0, 1])
+def test_plan_follows_the_instance(D, norm_only, bcast, weight):
     # scale and shift broadcast (stride_l 0) select the instances that re-read them from
     # cache, whose launch shape may differ; the plan reports the block the launch uses
-    h = make(D=D, gate=0 if norm_only else 1, norm_only=norm_only)
-    a = valid_args(D=D, B=1, L=1000, gate=not norm_only, norm_only=bool(norm_only))
+    h = make(D=D, gate=0 if norm_only else 1, norm_only=norm_only, weight=weight)
+    a = valid_args(D=D, B=1, L=1000, gate=not norm_only, weight=bool(weight), norm_only=bool(norm_only))
     if bcast:
         a.scale.stride_b = a.scale.stride_l = a.shift.stride_b = a.shift.stride_l = 0
     st, grid, block, smem = fn.fused_norm_plan(h, a)
     assert (st, grid, smem) == (OK, 1000, 0)
-    want = {(5120, False): 128, (10240, False): 320}[(D, False)]
-    if norm_only and bcast and D == 10240:
-        want = 256    # norm-only with cached modulation: 256 threads x 5 vectors
+    want = {5120: 128, 10240: 320}[D]
+    if norm_only and bcast:
+        # norm-only with cached modulation: 10 vectors per thread, except with an affine
+        # operand at D = 5120 (5 vectors)
+        want = 128 if (D == 5120 and weight) else D // 80
     assert block == want
 
 
