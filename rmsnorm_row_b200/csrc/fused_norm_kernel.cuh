@@ -359,8 +359,9 @@ __device__ __forceinline__ uint4 repair_vec(uint4 out, uint32_t near_mask, const
 // The same as one shared out-of-line copy. It runs for a few vectors in 10^3; in the
 // norm-only instances with 10 vectors per thread, one copy instead of one per unrolled
 // vector keeps the row loop's code small (instruction-fetch stalls 0.88 -> 0.24 per issue,
-// measured on B200: 2% faster). Where the kernel holds more live values, the call's
-// register saves cost more than that.
+// measured on B200: 2% faster without weight or bias; 3-7% with fp32 weight or bias at
+// D = 10240). Where the kernel holds more live values (the fused instances, norm-only with
+// bf16 weight or bias, fp32 ones at D = 5120), the call's register saves cost more (2-6%).
 template <bool HAS_WEIGHT, bool HAS_BIAS, class Affine>
 __device__ __noinline__ uint4 repair_vec_outlined(uint4 out, uint32_t near_mask, const uint4 v,
                                                   const uint4 sv, const uint4 tv, const Affine wf,
@@ -696,7 +697,7 @@ fused_norm_rows(const RowParams p) {
     using Affine = typename std::conditional<AFFINE_F32, AffineF32, AffineBF16>::type;
     const Affine wf = HAS_WEIGHT ? Affine::load(p.weight, j) : Affine::fill(1.0f);
     const Affine bf = HAS_BIAS ? Affine::load(p.bias, j) : Affine::fill(0.0f);
-    constexpr bool kOutlined = NORM_ONLY && CACHED_MOD && !HAS_WEIGHT && !HAS_BIAS;
+    constexpr bool kOutlined = NORM_ONLY && CACHED_MOD && ((!HAS_WEIGHT && !HAS_BIAS) || (D == 10240 && AFFINE_F32));
     __stcs(yo + j, output_vec<RowShape<D>::kPaired, kOutlined, HAS_WEIGHT, HAS_BIAS>(v[k], sv[k], tv[k], wf,
                                                                                    bf, st));
   }
