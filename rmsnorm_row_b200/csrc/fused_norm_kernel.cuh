@@ -36,6 +36,11 @@
 //     every row and stay in L1/L2). When scale and shift are both of the second kind,
 //     separate instances fetch them as each vector is used rather than holding them
 //     across the statistics, and run one more CTA per SM on the registers saved.
+//   * Norm-only rows with such scale and shift move 4 bytes per element, so their
+//     instruction count and the latency of each row's statistics set the pace: they
+//     hold 10 vectors per thread (fewer threads share each row's fixed work, more rows
+//     are in flight per SM) and, where it measured faster, call one shared out-of-line
+//     copy of the rare fp64 path instead of inlining it into every unrolled vector.
 #pragma once
 
 #include <cuda_bf16.h>
