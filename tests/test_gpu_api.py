@@ -10,6 +10,7 @@ on, that each call runs the CUDA kernel, and that one handle serves every launch
 * One handle launched with different L, frame counts and operand layouts matches the
   oracle bit for bit each time.
 * Launches captured into a CUDA graph replay to the eager results.
+* fused_norm_plan reports the grid and block that the launch uses, instance by instance.
 """
 import ctypes
 
@@ -187,3 +188,71 @@ def test_launches_replay_from_a_cuda_graph():
         for got, want in ((y, want_y), (r, want_r), (n, want_n)):
             assert torch.equal(got.view(torch.int16), want.view(torch.int16))
     del graph
+
+
+def _kernel_launches(prof, tmp_path):
+    """(name, grid, block) of each fused_norm_rows kernel in a profiler trace."""
+    import json
+    path = tmp_path / "trace.json"
+    prof.export_chrome_trace(str(path))
+    events = json.load(open(path)).get("traceEvents", [])
+    out = []
+    for e in events:
+        if e.get("cat") == "kernel" and "fused_norm_rows" in e.get("name", ""):
+            a = e.get("args", {})
+            if "grid" not in a or "block" not in a:
+                pytest.skip("the trace does not record launch dimensions")
+            out.append((e["name"], tuple(a["grid"]), tuple(a["block"])))
+    return out
+
+
+@pytest.mark.parametrize("D", [5120, 10240])
+@pytest.mark.parametrize("case", ["fused_row", "fused_bcast", "nss_bcast", "nss_bcast_w",
+                                  "nss_bcast_wb_f32", "nss_row"])
+def test_plan_matches_the_launch(D, case, tmp_path):
+    # the launch shape (threads per row) differs by instance; fused_norm_plan must report
+    # the grid and block the launch really uses, and the block must hold D / 8 vectors
+    # (the kernel's second template argument is the vectors per thread)
+    import re
+    from torch.profiler import ProfilerActivity, profile
+    dev = torch.device("cuda:0")
+    B, L = 1, 37
+    x = _rand((B, L, D), 41, dev)
+    norm_only = case.startswith("nss")
+    res = None if norm_only else _rand((B, L, D), 42, dev)
+    gate = None if norm_only else _rand((1, 1, D), 43, dev, 0.5)
+    per_row = case.endswith("_row")
+    shape = (B, L, D) if per_row else (1, 1, D)
+    scale, shift = _rand(shape, 44, dev, 0.1), _rand(shape, 45, dev, 0.1)
+    weight = bias = None
+    if case == "nss_bcast_w":
+        weight = (1 + _rand((D,), 46, dev, 0.1).float()).to(torch.bfloat16)
+    if case == "nss_bcast_wb_f32":
+        weight = 1 + _rand((D,), 46, dev, 0.1).float()
+        bias = _rand((D,), 47, dev, 0.1).float()
+    y = torch.empty_like(x)
+    r = None if norm_only else torch.empty_like(x)
+    args = fn.build_args(x, res, gate, weight, bias, scale, shift, y, r)
+    cfg = _abi.fn_config(D=D, is_rms=0, has_gate=int(gate is not None), has_weight=int(weight is not None),
+                         has_bias=int(bias is not None), norm_only=int(norm_only),
+                         affine_fp32=int(weight is not None and weight.dtype == torch.float32), eps=1e-6)
+    st, h = _abi.fused_norm_create(cfg)
+    assert st == fn.FN_OK
+    try:
+        st, grid, block, smem = _abi.fused_norm_plan(h, args)
+        assert st == fn.FN_OK and smem == 0
+        stream = int(torch.cuda.current_stream(dev).cuda_stream)
+        torch.cuda.synchronize(dev)
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            assert _abi.fused_norm_launch(h, args, stream) == fn.FN_OK
+            torch.cuda.synchronize(dev)
+        launches = _kernel_launches(prof, tmp_path)
+        if not launches:
+            pytest.skip("no CUDA activity recorded (tracing unavailable)")
+        assert len(launches) == 1, launches
+        name, g, b = launches[0]
+        assert g == (grid, 1, 1) and b == (block, 1, 1), (name, g, b, grid, block)
+        m = re.search(r"fused_norm_rows<(\d+), (\d+),", name)
+        assert m and int(m.group(1)) == D and block * 8 * int(m.group(2)) == D, name
+    finally:
+        _abi.fused_norm_destroy(h)
