@@ -58,6 +58,8 @@ MUTANTS = [
      "for (int64_t c = 0; c < D; ++c) mu = (double)(float)(mu + v[c]);", 0),
     ("variance_accumulated_in_float", "second += (v[c] - mu) * (v[c] - mu);",
      "second = (double)(float)(second + (v[c] - mu) * (v[c] - mu));", 0),
+    # a NaN statistic clamped away (fmax returns the non-NaN operand): NaN rows turn finite
+    ("nan_statistic_clamped", "1.0 / sqrt(second + eps)", "1.0 / sqrt(fmax(second, 0.0) + eps)", 0),
 ]
 
 
